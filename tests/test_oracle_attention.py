@@ -1,0 +1,149 @@
+"""Pins for the oracle's mixed-precision attention (CPU).
+
+* a 0/0/0/100 budget must give dense softmax attention (torch's fp64
+  scaled_dot_product_attention is the reference), padding included;
+* a partial 16-bit budget must give dense attention restricted to the kept
+  key blocks (a boolean mask on the same library routine);
+* a 100 % skip budget gives zeros;
+* Q = 0 makes every score equal, which fixes the low-bit phases in closed form;
+* a single-precision low-bit budget stays within the error bound that P's
+  quantisation alone allows, against exact attention on the dequantised
+  operands;
+* emulate mode differs from math mode only by bf16 rounding.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, formats as F, geometry, pipeline, prep
+from oracle.problem import Problem
+from mixed_precision_block_b200.synth import Workload, make_qkv
+
+
+def _inputs(T=2, Hh=12, Ww=10, d=32, H=1, seed=0, budget=(0, 0, 0, 100), lam=0.5):
+    wl = Workload("t", 1, H, T, Hh, Ww, d, lam, budget, seed=seed)
+    q, k, v = make_qkv(wl)
+    p = Problem.from_workload(wl)
+    return p, pipeline.to_f64(q)[0, 0], pipeline.to_f64(k)[0, 0], pipeline.to_f64(v)[0, 0]
+
+
+def _sdpa(q, k, v, mask=None):
+    t = [torch.from_numpy(x)[None, None] for x in (q, k, v)]
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(*t, attn_mask=m)[0, 0].numpy()
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / np.linalg.norm(b)
+
+
+def test_full_16bit_budget_is_dense_attention():
+    p, q, k, v = _inputs()
+    r = pipeline.run_head(p, q, k, v, mode="math")
+    assert _rel(r["out"], _sdpa(q, k, v)) < 1e-13
+    r = pipeline.run_head(p, q, k, v, mode="emulate")
+    assert 1e-4 < _rel(r["out"], _sdpa(q, k, v)) < 4e-3  # bf16 P and output
+
+
+def test_partial_16bit_budget_is_masked_dense_attention():
+    p, q, k, v = _inputs(budget=(60, 0, 0, 40))
+    r = pipeline.run_head(p, q, k, v, mode="math")
+    tab = r["prep"]["table"]
+    keep = r["map"] == 16
+    # token-level mask from the block-level assignment
+    tok_blk = np.zeros(p.N, dtype=np.int64)
+    for b in range(p.nb):
+        tok_blk[tab[b][tab[b] >= 0]] = b
+    mask = keep[tok_blk][:, tok_blk]
+    want = _sdpa(q, k, v, mask)
+    rows = mask.any(1)
+    assert rows.all()  # this budget leaves no query region empty here
+    assert _rel(r["out"], want) < 1e-13
+
+
+def test_all_skipped_gives_zeros():
+    p, q, k, v = _inputs(budget=(100, 0, 0, 0))
+    r = pipeline.run_head(p, q, k, v, mode="emulate")
+    assert not r["out"].any()
+
+
+def test_q_zero_closed_forms():
+    p, q, k, v = _inputs(Hh=12, Ww=10)
+    q = np.zeros_like(q)
+    # 8-bit only: every score 0 → p = 1 → code 255 → mean of the INT8-dequantised V
+    p8 = Problem(**{**p.__dict__, "budget": (0, 0, 100, 0)})
+    r = pipeline.run_head(p8, q, k, v, mode="math")
+    vb = r["prep"]["v_i8"].astype(np.float64) * r["prep"]["v_s8"][None, :, None]  # [nb, d, S]
+    vt = np.concatenate([vb[b][:, r["prep"]["valid"][b]] for b in range(p.nb)], axis=1)
+    np.testing.assert_allclose(r["out"], np.broadcast_to(vt.mean(1), r["out"].shape), rtol=1e-12)
+    # 4-bit only: p = 1 → sf = e4m3(1/6) = 0.171875, code e2m1(5.818) = 6 → weight 1.03125
+    assert F.e4m3_round(1.0 / 6.0) == 0.171875
+    p4 = Problem(**{**p.__dict__, "budget": (0, 100, 0, 0)})
+    r = pipeline.run_head(p4, q, k, v, mode="math")
+    pr = r["prep"]
+    vd = prep.dequant_v_nvfp4(pr["v_f4"], pr["v_sf4"], pr["v_g4"])
+    vt = np.concatenate([vd[b][:, pr["valid"][b]] for b in range(p.nb)], axis=1)
+    np.testing.assert_allclose(r["out"], np.broadcast_to(1.03125 * vt.mean(1), r["out"].shape), rtol=1e-12)
+
+
+def _dequant_dense(p, pr, fmt):
+    """Token-order dequantised Q, K, V of one head for the given phase format."""
+    tab = pr["table"]
+    valid = tab >= 0
+    if fmt == 8:
+        qd = pr["q_i8"] * pr["q_s8"][:, None, None]
+        kd = pr["k_i8"] * pr["k_s8"][:, None, None]
+        vd = (pr["v_i8"] * pr["v_s8"][None, :, None]).transpose(0, 2, 1)
+    else:
+        qd = F.nvfp4_dequantize(pr["q_f4"], pr["q_sf4"])
+        kd = F.nvfp4_dequantize(pr["k_f4"], pr["k_sf4"])
+        vd = prep.dequant_v_nvfp4(pr["v_f4"], pr["v_sf4"], pr["v_g4"]).transpose(0, 2, 1)
+    out = []
+    for x in (qd, kd, vd):
+        y = np.zeros((p.N, p.d))
+        y[tab[valid]] = x[valid]
+        out.append(y)
+    return out
+
+
+@pytest.mark.parametrize("fmt", [8, 4])
+def test_low_bit_phase_within_p_quantisation_bound(fmt):
+    budget = (0, 0, 100, 0) if fmt == 8 else (0, 100, 0, 0)
+    p, q, k, v = _inputs(Hh=12, Ww=10, budget=budget)
+    r = pipeline.run_head(p, q, k, v, mode="math")
+    qd, kd, vd = _dequant_dense(p, r["prep"], fmt)
+    exact = _sdpa(qd, kd, vd)
+    # bound: each weight's error is at most e * exp(m_blk - m) / l, e the
+    # largest rounding error of one quantised p in (0, 1] relative to its block max
+    # (INT8: half a step of 1/255; NVFP4: the sf step plus saturation, < 0.18)
+    e = 0.5 / 255 if fmt == 8 else 0.18
+    s = qd @ kd.T / np.sqrt(p.d)
+    tab = r["prep"]["table"]
+    m = s.max(1)
+    l = np.exp(s - m[:, None]).sum(1)
+    bound = np.zeros((p.N, p.d))
+    for b in range(p.nb):
+        toks = tab[b][tab[b] >= 0]
+        mb = s[:, toks].max(1)
+        bound += (e * np.exp(mb - m) / l)[:, None] * np.abs(vd[toks]).sum(0)[None, :]
+    err = np.abs(r["out"] - exact)
+    assert err.max() > 0
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-12)
+    # and the phase stays close to exact attention on its own operands
+    assert _rel(r["out"], exact) < (0.01 if fmt == 8 else 0.06)
+
+
+def test_emulate_is_math_plus_bf16_rounding():
+    p, q, k, v = _inputs(budget=(10, 40, 50, 0))
+    a = pipeline.run_head(p, q, k, v, mode="math")["out"]
+    b = pipeline.run_head(p, q, k, v, mode="emulate")["out"]
+    np.testing.assert_array_equal(b, attention.bf16_round(a))
+
+
+def test_scatter_restores_token_order():
+    p = Problem(1, 1, 2, 10, 13, 4, 0.5, (0, 0, 0, 100))
+    tab = geometry.block_tokens(p)
+    x = np.random.default_rng(0).standard_normal((p.N, 4))
+    blocks, _ = prep.gather_blocks(x, tab)
+    np.testing.assert_array_equal(attention.scatter(blocks, tab, p.N), x)
