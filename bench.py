@@ -1,0 +1,387 @@
+"""Benchmark of one DraftAttention2 attention call on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload video] [--impl ours|reference]
+
+A step is one whole call — da2_prepare (reorder, pool, quantise), da2_draft_rank
+(draft map, ranking, assignment) and da2_attention (mixed-precision attention,
+output restored to token order) — on the 118,800-token (33x45x80 latent),
+24-head, d=128 bf16 workload with budget skip/4/8/16 = 85/0/7.5/7.5 and
+lambda = 0.5, seeded synthetic blob + noise + outlier inputs resident in HBM.
+Each input tensor (730 MB) is larger than L2, so no flush is needed.
+
+Printed on rank 0, one JSON line: effective (dense-equivalent) TFLOP/s of the
+whole job, ms per call, the roofline of the attention kernel, the own dense
+bf16 kernel on the same inputs, an end-to-end figure through host buffers,
+SM clocks sampled during the timed region, and the CPU oracle as a reported
+baseline.  ``--impl reference`` times the CPU oracle alone (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "attention-call ms + effective TFLOP/s (118.8K tok, 24 heads) vs own dense bf16"
+UNIT = "TFLOP/s (dense-equivalent)"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAK_FALLBACK, "fallback"
+
+
+def phase_flops(wl, info):
+    """Executed MMA FLOPs per phase: 4 * 64 * 64 * d per retained block pair."""
+    per_pair = 4.0 * 64 * 64 * wl.d
+    bh = wl.B * wl.H
+    return {16: per_pair * info.n16 * bh, 8: per_pair * info.n8 * bh, 4: per_pair * info.n4 * bh}
+
+
+def launches_per_call(info):
+    """Kernels this library launches per call (its own kernels only)."""
+    v = 2 if (info.n8 or info.n4) else 0  # v_amax + pack_v
+    prep = 1 + v
+    draft = 2  # logits + mix (mix carries the first ranking histogram)
+    rank = 1 + 8 + 7 + 1  # init, 8 selects, 7 histogram passes, assign
+    return prep + draft + rank + 1
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        else:
+            self.lines = []
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except (ValueError, IndexError):
+                continue
+            for n, val in zip(names, f[3:7]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"]}
+        # samples under load: the upper half of the readings
+        load = sorted(sm)[len(sm) // 2:]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_sample(wl, frames=4, seed=0):
+    """Time the CPU oracle on a bounded sample and extrapolate to one whole call.
+
+    The sample is the same workload cut to its first ``frames`` latent frames
+    and one head (same grid, regions, d, budget, lambda), run through every
+    stage in full.  Each stage is scaled to the full workload by its own
+    complexity: prep by tokens, draft by region pairs, ranking by pairs x
+    log(pairs), attention by kept block pairs, and all by the head count.
+    Returns (seconds per call, cores, description)."""
+    import math
+    import numpy as np
+    import torch
+    from oracle import draft as ODR, geometry as OG, prep as OP, rank as OR, attention as OA
+    from oracle.problem import Problem as OProblem
+    from mixed_precision_block_b200.synth import make_qkv
+
+    small = wl.with_(H=1, B=1, T=min(frames, wl.T))
+    q, k, v = make_qkv(small, "cpu", seed=seed)
+    op = OProblem.from_workload(small)
+    full = OProblem.from_workload(wl)
+    qh, kh, vh = (x[0, 0].float().numpy().astype(np.float64) for x in (q, k, v))
+    t0 = time.perf_counter()
+    table = OG.block_tokens(op)
+    pr = OP.prepare_head(op, qh, kh, vh, table)
+    t1 = time.perf_counter()
+    D = ODR.draft_scores(pr["q_avg"], pr["k_avg"], pr["q_max"], pr["k_max"], op.lam, op.d)
+    t2 = time.perf_counter()
+    n16, n8, n4, _ = OG.budget_counts(op)
+    pmap = OR.assign(D, n16, n8, n4)
+    t3 = time.perf_counter()
+    OA.head_attention(pr, pmap, op.d, "emulate")
+    t4 = time.perf_counter()
+    P_s, P_f = op.nb ** 2, full.nb ** 2
+    f16, f8, f4, _ = OG.budget_counts(full)
+    kept_s, kept_f = n16 + n8 + n4, f16 + f8 + f4
+    head_s = ((t1 - t0) * full.N / op.N + (t2 - t1) * P_f / P_s
+              + (t3 - t2) * (P_f * math.log(P_f)) / (P_s * math.log(P_s))
+              + (t4 - t3) * kept_f / max(kept_s, 1))
+    call_s = head_s * wl.B * wl.H
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = torch.get_num_threads()
+    desc = (f"oracle (numpy fp64) on 1 head of the first {small.T} of {wl.T} frames "
+            f"({op.N} tokens, {op.nb} regions): prep {t1 - t0:.2f} s, draft {t2 - t1:.2f} s, "
+            f"rank {t3 - t2:.2f} s, attention {t4 - t3:.2f} s; scaled per stage by tokens, pairs, "
+            f"pairs*log(pairs), kept pairs, and x{wl.B * wl.H} heads")
+    return call_s, cores, desc
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from mixed_precision_block_b200.synth import dense_flops
+    flops = dense_flops(wl)
+    times, cores, desc = [], 1, ""
+    for i in range(args.warmup + args.steps):
+        s, cores, desc = cpu_oracle_sample(wl, frames=args.ref_frames, seed=i)
+        if i >= args.warmup:
+            times.append(s)
+    sec = statistics.mean(times)
+    val = flops / sec / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, args),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args):
+    return {"workload": f"{wl.name}: B={wl.B} H={wl.H} grid {wl.T}x{wl.Hh}x{wl.Ww} "
+                        f"({wl.N} tokens) d={wl.d} regions {wl.rh}x{wl.rw}",
+            "budget_skip_4_8_16": list(wl.budget), "lambda": wl.lam, "seed": wl.seed,
+            "inputs": "bf16 blob+noise+outlier, each tensor larger than L2 (no flush)",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def traffic_record(kernel_src):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None if the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "attn_mp_video_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return rec.get("dram_bytes_per_launch") if rec.get("source_sha256") == h else None
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+    from mixed_precision_block_b200 import da2
+    from mixed_precision_block_b200.synth import make_qkv, dense_flops
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    q, k, v = make_qkv(wl, dev)
+    p = da2.Problem.from_workload(wl)
+    info = da2.da2_plan(p)
+    ws = da2.workspace(p, dev)
+    out = torch.empty_like(q)
+    st = torch.cuda.Stream(dev)
+    flops = dense_flops(wl)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        da2.da2_prepare(p, q, k, v, ws, st)
+        if ev is not None:
+            ev[1].record(st)
+        da2.da2_draft_rank(p, ws, st)
+        if ev is not None:
+            ev[2].record(st)
+        da2.da2_attention(p, q, k, v, ws, out, st)
+        if ev is not None:
+            ev[3].record(st)
+
+    with torch.cuda.stream(st):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(st)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(st)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    stage = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # own dense bf16 kernel on the same inputs
+    dense_out = torch.empty_like(q)
+    with torch.cuda.stream(st):
+        da2.da2_dense_attention(q, k, v, dense_out, st)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(st)
+        for _ in range(args.dense_steps):
+            da2.da2_dense_attention(q, k, v, dense_out, st)
+        d1.record(st)
+    torch.cuda.synchronize(dev)
+    dense_ms = d0.elapsed_time(d1) / args.dense_steps
+
+    # end to end through host buffers: pinned H2D of Q/K/V, the call, D2H of O
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            da2.attention(p, dq, dk, dv, ws, out, st)
+            hout.copy_(out, non_blocking=True)
+
+        with torch.cuda.stream(st):
+            e2e_step()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(st)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            a1.record(st)
+        torch.cuda.synchronize(dev)
+        e_ms = a0.elapsed_time(a1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+        del hq, hk, hv, hout, dq, dk, dv
+
+    pk, pk_kind = peaks()
+    sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    pf = phase_flops(wl, info)
+    f_tot = sum(pf.values())
+    t_roof_s = pf[16] / (sus * 1e12) + pf[8] / (2 * sus * 1e12) + pf[4] / (4 * sus * 1e12)
+    attn_ms = stage[2]
+    achieved = f_tot / (attn_ms * 1e-3) / 1e12
+    peak_blend = f_tot / t_roof_s / 1e12
+    traffic = traffic_record(os.path.join(ROOT, "mixed_precision_block_b200", "csrc", "attn.cu"))
+    clocks = clk.summary()
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu:
+            s, cores, desc = cpu_oracle_sample(wl, frames=args.cpu_frames)
+            cpu = {"value": flops / s / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16+int8+nvfp4 (fp32 accumulate)", "data": "synthetic",
+            "config": config_of(wl, args),
+            "stages_ms": {"prepare": stage[0], "draft_rank": stage[1], "attention": stage[2]},
+            "dense_bf16": {"ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
+                           "speedup_of_sparse_call": dense_ms / ms},
+            "roofline": {"bound": "tensor", "kernel": "attn_mp_kernel", "achieved": achieved,
+                         "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
+                         "traffic": traffic,
+                         "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
+                                      f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
+                                      f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"},
+            "e2e": e2e, "gpu_launches": launches_per_call(info) * args.steps, "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="video")
+    ap.add_argument("--lam", type=float, default=None)
+    ap.add_argument("--dense-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-frames", type=int, default=2, help="frames per CPU oracle sample (reference arm)")
+    ap.add_argument("--cpu-frames", type=int, default=8, help="frames of the CPU-baseline oracle sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # fewer warm-up steps would not give a valid number
+    from mixed_precision_block_b200.synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.lam is not None:
+        wl = wl.with_(lam=args.lam)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

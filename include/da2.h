@@ -1,0 +1,159 @@
+/*
+ * da2.h — C ABI of libda2.so, a B200 (sm_100a) implementation of the
+ * DraftAttention2 low-resolution-guided mixed-precision block-sparse attention.
+ *
+ * Sources, cited by page title and section:
+ *   [abstract]  DraftAttention2: Fast Video Diffusion with Low-Resolution-Guided
+ *               Mixed-Precision Attention — Abstract.
+ *   [note]      DraftAttention2 reading note (Chinese blog post on the same
+ *               paper) — "Method overview" bullets 1-4, Figure 2 and Figure 3
+ *               captions, experiment section.
+ *   [v1]        DraftAttention: Fast Video Diffusion via Low-Resolution
+ *               Attention Guidance — Abstract.
+ *
+ * One attention call is three entry points enqueued on one stream:
+ *   da2_prepare     reorder Q/K/V into region blocks, pool, quantise
+ *   da2_draft_rank  draft map, shared per-head ranking, precision assignment
+ *   da2_attention   mixed-precision attention, output restored to token order
+ *
+ * Conventions (all entry points):
+ *   - Q, K, V and the output are bf16, contiguous [B, H, N, d] with
+ *     N = T*Hh*Ww and token n = (t*Hh + y)*Ww + x; device pointers, 16-byte
+ *     aligned.  The caller owns every buffer.
+ *   - `ws` is a caller-allocated device workspace of at least
+ *     da2_plan_info.ws_bytes bytes (256-byte aligned); it carries the prepared
+ *     operands and the assignment from one call to the next, so the three calls
+ *     of one attention must use the same workspace and problem.  The library
+ *     allocates no device memory and keeps no state between calls beyond
+ *     per-device function attributes; calls with distinct workspaces may run
+ *     concurrently on different streams.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All device work is asynchronous on that stream.
+ *   - Return value: DA2_OK or an error code; nothing throws across the ABI.
+ *     Argument errors are detected on the host before any launch.  A launch
+ *     failure returns DA2_ERR_CUDA.
+ */
+#ifndef DA2_H
+#define DA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DA2_OK = 0,
+  DA2_ERR_ARG = 1,          /* invalid sizes, pointers, lambda or budget       */
+  DA2_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, rh*rw != 64, no sm_100 GPU    */
+  DA2_ERR_WORKSPACE = 3,    /* workspace NULL, misaligned or too small         */
+  DA2_ERR_CUDA = 4          /* a CUDA launch or runtime call failed            */
+};
+
+/* Problem statement of one attention call.
+ * Region size rh x rw cuts every frame's Hh x Ww grid into regions; frames are
+ * padded to multiples of the region size and padding tokens are masked
+ * ([note] Figure 3(a)).  rh*rw must be 64 (one region = one 64-token block).
+ * lambda in [0,1] weights the max-pooled draft map ([note] Method overview
+ * bullet 1; lambda = 0 is average-only drafting, [v1]).
+ * budget_pct = {skip, 4-bit, 8-bit, 16-bit} percentages of the region pairs of
+ * each head ([note] experiment section, "Bit" column 0/4/8/16).  The 4/8/16
+ * shares must be >= 0 with sum <= 100; the four must sum to 100 within 0.2
+ * (published budgets are rounded, e.g. 80.7/14.4/4.8/0); skip is taken as the
+ * remainder. */
+typedef struct da2_problem {
+  int B, H, T, Hh, Ww, d;
+  int rh, rw;
+  float lambda;
+  float budget_pct[4];
+} da2_problem;
+
+/* Derived sizes.  Counts are per (batch, head): with P = nb^2 pairs and
+ * permille shares q = round(10*pct), cumulative counts c = floor((P*cum+500)/1000)
+ * taken in order 16, 8, 4. */
+typedef struct da2_plan_info {
+  long long pairs_per_head;
+  long long n16, n8, n4, nskip;
+  int nb, nry, nrx, N, Np;
+  size_t ws_bytes;
+} da2_plan_info;
+
+/* Validates `p` and fills `out`.  Host only, no device work. */
+int da2_plan(const da2_problem* p, da2_plan_info* out);
+
+/* Stage 1 ([abstract]; [note] Method overview bullet 4, Figure 3(b)).
+ * Per (batch, head, region block): the block's 64 tokens are gathered from
+ * Q and K, their average and channel-wise max descriptors are pooled over the
+ * region's real tokens, and Q/K are quantised to INT8 (one fp32 scale per
+ * block) and NVFP4 (e4m3 scale per 16 channels of a token).  V is quantised
+ * per channel (INT8; NVFP4 with a per-channel fp32 scale and e4m3 scales per
+ * 16 tokens) and transposed to [block][channel][token].  Formats the budget
+ * does not use are not written.  q, k, v: device bf16 [B,H,N,d]. */
+int da2_prepare(const da2_problem* p, const void* q, const void* k, const void* v,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 2 ([abstract]; [note] Method overview bullets 1-2, Figure 2).
+ * Draft map D = (1-lambda)*softmax(avgQ avgK^T/sqrt d) + lambda*softmax(maxQ maxK^T/sqrt d)
+ * per head over region pairs (fp32), then one ranking per head, descending by D
+ * with ties broken by ascending pair index q_block*nb + k_block, hands out the
+ * budget: first n16 pairs 16-bit, next n8 INT8, next n4 NVFP4, rest skipped.
+ * Requires da2_prepare on the same workspace first. */
+int da2_draft_rank(const da2_problem* p, void* ws, size_t ws_bytes, void* stream);
+
+/* Test hook for stage 2: ranking and assignment only, on caller-given fp32
+ * scores [B,H,nb,nb] (device), which are copied into the workspace first. */
+int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Stage 3 ([abstract]; [note] Method overview bullet 4; [v1] order restore).
+ * Per query block one pass runs the 16-bit phase (bf16 Q/K/V), the INT8 phase
+ * and the NVFP4 phase over its assigned key blocks with one shared online
+ * softmax state and one fp32 accumulator; low-bit P is quantised relative to
+ * each key block's row maximum; quantisation scales are applied when a block
+ * is merged.  The output rows are written straight back to the original token
+ * order (padding rows dropped); a query block with no key block outputs zeros.
+ * q, k, v: the same device tensors given to da2_prepare; out: device bf16
+ * [B,H,N,d].  Requires da2_draft_rank (or da2_rank_from_scores) first. */
+int da2_attention(const da2_problem* p, const void* q, const void* k, const void* v,
+                  void* ws, size_t ws_bytes, void* out, void* stream);
+
+/* Own dense bf16 softmax attention over all N tokens (the comparison point
+ * for the sparse path): out = softmax(q k^T / sqrt d) v, fp32 accumulation,
+ * bf16 output.  q, k, v, out: device bf16 [B,H,N,d]; d in {64,128}. */
+int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k,
+                        const void* v, void* out, void* stream);
+
+/* Workspace views for tests.  Returns the device address and size of one
+ * intermediate inside `ws` (no device work).  Layouts (bh = b*H + h):
+ *   PERM   int32 [nb][64]            token of each block slot, -1 = padding
+ *   Q_AVG/K_AVG/Q_MAX/K_MAX  fp32 [B*H][nb][d]
+ *   Q_I8/K_I8  int8 [B*H][nb][64][d];  Q_S8/K_S8 fp32 [B*H][nb]
+ *   Q_F4/K_F4  uint8 [B*H][nb][64][d/2] (even channel in the low nibble)
+ *   Q_SF4/K_SF4 uint8 e4m3 [B*H][nb][64][d/16]
+ *   V_I8  int8 [B*H][nb][d][64];  V_S8 fp32 [B*H][d]
+ *   V_F4  uint8 [B*H][nb][d][32] (even token in the low nibble)
+ *   V_SF4 uint8 e4m3 [B*H][nb][d][4];  V_G4 fp32 [B*H][d]
+ *   SCORES fp32 [B*H][nb][nb]
+ *   MAP    uint8 [B*H][nb][nb]  precision per pair: 16, 8, 4 or 0 (skip)
+ *   LISTS  uint16 [B*H][nb][nb] per query block: its 16-bit key blocks, then
+ *          its 8-bit, then its 4-bit ones, each ascending
+ *   COUNTS int32 [B*H][nb][4]   lengths of the three lists, 0 */
+enum {
+  DA2_VIEW_PERM = 0,
+  DA2_VIEW_Q_AVG, DA2_VIEW_K_AVG, DA2_VIEW_Q_MAX, DA2_VIEW_K_MAX,
+  DA2_VIEW_Q_I8, DA2_VIEW_K_I8, DA2_VIEW_Q_S8, DA2_VIEW_K_S8,
+  DA2_VIEW_Q_F4, DA2_VIEW_K_F4, DA2_VIEW_Q_SF4, DA2_VIEW_K_SF4,
+  DA2_VIEW_V_I8, DA2_VIEW_V_S8, DA2_VIEW_V_F4, DA2_VIEW_V_SF4, DA2_VIEW_V_G4,
+  DA2_VIEW_SCORES, DA2_VIEW_MAP, DA2_VIEW_LISTS, DA2_VIEW_COUNTS,
+  DA2_VIEW_COUNT_
+};
+int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes);
+
+/* Human-readable name of a status code (static string). */
+const char* da2_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DA2_H */

@@ -1,0 +1,183 @@
+// C-ABI entry points of libda2.so: argument validation, geometry, workspace
+// layout, and the launch sequence of each stage.  See include/da2.h.
+#include <cmath>
+#include <cstring>
+
+#include "da2_internal.cuh"
+
+using namespace da2;
+
+namespace {
+
+int permille(float pct) { return (int)std::lrint(10.0 * (double)pct); }
+
+int check_device() {
+  static int cached[64];  // 0 = unknown, 1 = ok, 2 = unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DA2_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return DA2_ERR_UNSUPPORTED;
+  if (cached[dev] == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return DA2_ERR_CUDA;
+    cached[dev] = (major == 10) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? DA2_OK : DA2_ERR_UNSUPPORTED;
+}
+
+int make_geom(const da2_problem* p, Geom* g) {
+  if (!p || !g) return DA2_ERR_ARG;
+  if (p->B <= 0 || p->H <= 0 || p->T <= 0 || p->Hh <= 0 || p->Ww <= 0) return DA2_ERR_ARG;
+  if (p->rh <= 0 || p->rw <= 0) return DA2_ERR_ARG;
+  if (p->d != 64 && p->d != 128) return DA2_ERR_UNSUPPORTED;
+  if (p->rh * p->rw != kBlockTokens) return DA2_ERR_UNSUPPORTED;
+  if (!(p->lambda >= 0.f && p->lambda <= 1.f)) return DA2_ERR_ARG;
+  double sum = 0;
+  for (int i = 0; i < 4; ++i) {
+    if (!(p->budget_pct[i] >= 0.f) || !(p->budget_pct[i] <= 100.f)) return DA2_ERR_ARG;
+    sum += p->budget_pct[i];
+  }
+  if (std::fabs(sum - 100.0) > 0.2) return DA2_ERR_ARG;
+  const int q4 = permille(p->budget_pct[1]), q8 = permille(p->budget_pct[2]),
+            q16 = permille(p->budget_pct[3]);
+  if (q4 + q8 + q16 > 1000) return DA2_ERR_ARG;
+  g->B = p->B; g->H = p->H; g->T = p->T; g->Hh = p->Hh; g->Ww = p->Ww; g->d = p->d;
+  g->rh = p->rh; g->rw = p->rw;
+  g->nry = (p->Hh + p->rh - 1) / p->rh;
+  g->nrx = (p->Ww + p->rw - 1) / p->rw;
+  const long long nb = (long long)p->T * g->nry * g->nrx;
+  const long long N = (long long)p->T * p->Hh * p->Ww;
+  if (nb > 65535 || N > (1LL << 30) || (long long)p->B * p->H > (1LL << 20)) return DA2_ERR_UNSUPPORTED;
+  g->nb = (int)nb;
+  g->N = (int)N;
+  g->BH = p->B * p->H;
+  g->lambda = p->lambda;
+  const long long P = nb * nb;
+  auto cnt = [&](int cum) { return (P * cum + 500) / 1000; };
+  const long long c16 = cnt(q16), c8 = cnt(q16 + q8), c4 = cnt(q16 + q8 + q4);
+  g->n16 = c16; g->n8 = c8 - c16; g->n4 = c4 - c8;
+  g->cut[0] = c16; g->cut[1] = c8; g->cut[2] = c4;
+  return DA2_OK;
+}
+
+int check_ws(const Layout& L, const void* ws, size_t ws_bytes) {
+  if (!ws || ((uintptr_t)ws & 255) != 0) return DA2_ERR_WORKSPACE;
+  if (ws_bytes < L.total) return DA2_ERR_WORKSPACE;
+  return DA2_OK;
+}
+
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int da2_plan(const da2_problem* p, da2_plan_info* out) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!out) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  out->pairs_per_head = (long long)g.nb * g.nb;
+  out->n16 = g.n16; out->n8 = g.n8; out->n4 = g.n4;
+  out->nskip = out->pairs_per_head - g.cut[2];
+  out->nb = g.nb; out->nry = g.nry; out->nrx = g.nrx; out->N = g.N;
+  out->Np = g.nb * kBlockTokens;
+  out->ws_bytes = L.total;
+  return DA2_OK;
+}
+
+int da2_prepare(const da2_problem* p, const void* q, const void* k, const void* v,
+                void* ws, size_t ws_bytes, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  if ((rc = check_ws(L, ws, ws_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  return cuda_status(launch_prepare(g, L, q, k, v, ws, (cudaStream_t)stream));
+}
+
+int da2_draft_rank(const da2_problem* p, void* ws, size_t ws_bytes, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  const Layout L = make_layout(g);
+  if ((rc = check_ws(L, ws, ws_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = launch_draft(g, L, ws, st);
+  if (e == cudaSuccess) e = launch_rank(g, L, ws, /*hist0_done=*/true, st);
+  return cuda_status(e);
+}
+
+int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!aligned16(scores)) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  if ((rc = check_ws(L, ws, ws_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(at<float>(ws, L, R_SCORES), scores, L.size[R_SCORES],
+                                  cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = launch_rank(g, L, ws, /*hist0_done=*/false, st);
+  return cuda_status(e);
+}
+
+int da2_attention(const da2_problem* p, const void* q, const void* k, const void* v,
+                  void* ws, size_t ws_bytes, void* out, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  if ((rc = check_ws(L, ws, ws_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  return cuda_status(launch_attention(g, L, q, k, v, ws, out, (cudaStream_t)stream));
+}
+
+int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k,
+                        const void* v, void* out, void* stream) {
+  if (B <= 0 || H <= 0 || N <= 0) return DA2_ERR_ARG;
+  if (d != 64 && d != 128) return DA2_ERR_UNSUPPORTED;
+  if ((long long)B * H > (1LL << 20) || N > (1 << 30)) return DA2_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DA2_ERR_ARG;
+  int rc = check_device();
+  if (rc) return rc;
+  return cuda_status(launch_dense(B, H, N, d, q, k, v, out, (cudaStream_t)stream));
+}
+
+int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!ws || !ptr || !bytes) return DA2_ERR_ARG;
+  static const Region map[DA2_VIEW_COUNT_] = {
+      R_PERM, R_Q_AVG, R_K_AVG, R_Q_MAX, R_K_MAX, R_Q_I8, R_K_I8, R_Q_S8, R_K_S8,
+      R_Q_F4, R_K_F4, R_Q_SF4, R_K_SF4, R_V_I8, R_V_S8, R_V_F4, R_V_SF4, R_V_G4,
+      R_SCORES, R_MAP, R_LISTS, R_COUNTS};
+  if (which < 0 || which >= DA2_VIEW_COUNT_) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  *ptr = static_cast<char*>(ws) + L.off[map[which]];
+  *bytes = L.size[map[which]];
+  return DA2_OK;
+}
+
+const char* da2_status_string(int s) {
+  switch (s) {
+    case DA2_OK: return "ok";
+    case DA2_ERR_ARG: return "invalid argument";
+    case DA2_ERR_UNSUPPORTED: return "unsupported problem or device";
+    case DA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DA2_ERR_CUDA: return "CUDA launch or runtime error";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,337 @@
+// Stage 1: fused operand preparation.
+//
+// DraftAttention2 abstract and reading note (Method overview bullet 4,
+// Figure 3(b)): Q/K reordering, pooling and quantisation share one kernel;
+// V is reordered and transposed while it is packed.
+//
+// prep_qk: one CTA per (region block, head, tensor Q|K).  The block's 64 tokens
+//   are 8 rows of 8 consecutive tokens in the [B,H,N,d] input, so each token
+//   is one contiguous d*2-byte row; 256 threads read it in 16-byte chunks
+//   (coalesced 128-bit loads, padding slots are never read).  In one pass the
+//   CTA produces the pooled mean / max (warp-shuffle + shared-memory
+//   reductions), the INT8 codes with the block's absmax scale, and the NVFP4
+//   codes with one e4m3 scale per 16 channels of a token.
+// v_amax + pack_v: the per-channel absmax of V over all real tokens of a head
+//   (first pass, atomicMax on the float bits), then one CTA per block that
+//   stages the block transposed in shared memory and writes INT8 and NVFP4
+//   codes in [block][channel][token] order.
+#include "da2_internal.cuh"
+
+namespace da2 {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct PrepPtrs {
+  const __nv_bfloat16* x[2];
+  float* avg[2];
+  float* mx[2];
+  int8_t* i8[2];
+  float* s8[2];
+  uint8_t* f4[2];
+  uint8_t* sf4[2];
+  int* perm;
+};
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Number of real tokens in a region block.
+__device__ __forceinline__ int block_real_count(const Geom& g, int blk) {
+  const int rx = blk % g.nrx;
+  const int ry = (blk / g.nrx) % g.nry;
+  const int ny = min(g.rh, g.Hh - ry * g.rh);
+  const int nx = min(g.rw, g.Ww - rx * g.rw);
+  return ny * nx;
+}
+
+__device__ __forceinline__ uint32_t quant_i8x4(const float* x, float inv) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int c = __float2int_rn(__fmul_rn(x[i], inv));
+    c = max(-127, min(127, c));
+    r |= (uint32_t)(c & 0xff) << (8 * i);
+  }
+  return r;
+}
+
+// NVFP4 microblock of 16 values held as 8 per lane in lanes (2j, 2j+1):
+// returns 4 code bytes for this lane's 8 values and the e4m3 scale byte.
+__device__ __forceinline__ uint32_t quant_f4x8(const float* x, float amax16, uint32_t* sf_byte) {
+  const float t = __fdiv_rn(amax16, 6.0f);
+  const uint32_t sf = cvt_e4m3x2(0.0f, t) & 0xffu;
+  *sf_byte = sf;
+  const float dec = e4m3_to_f32(sf);
+  if (dec == 0.0f) return 0u;
+  const float r = __fdiv_rn(1.0f, dec);
+  uint32_t out = 0;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t b = cvt_e2m1x2(__fmul_rn(x[2 * m + 1], r), __fmul_rn(x[2 * m], r));
+    out |= b << (8 * m);
+  }
+  return out;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) prep_qk_kernel(Geom g, PrepPtrs P, int want_i8,
+                                                           int want_f4) {
+  constexpr int CPT = D / 8;                // 16-byte chunks per token
+  constexpr int NC = 64 * CPT / kThreads;   // chunks per thread
+  constexpr int SLOT_STEP = kThreads / CPT;
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid % CPT, slot0 = tid / CPT;
+  const __nv_bfloat16* __restrict__ x = P.x[which] + (size_t)bh * g.N * D;
+
+  float v[NC][8];
+  bool valid[NC];
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int s = slot0 + i * SLOT_STEP;
+    const int tok = slot_token(g, blk, s);
+    valid[i] = tok >= 0;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (valid[i]) u = *reinterpret_cast<const uint4*>(x + (size_t)tok * D + cg * 8);
+    unpack8(u, v[i]);
+  }
+  if (which == 0 && bh == 0 && tid < 64) P.perm[blk * 64 + tid] = slot_token(g, blk, tid);
+
+  // ---- pooled mean and max over real tokens
+  float psum[8], pmax[8], amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) { psum[c] = 0.f; pmax[c] = -INFINITY; }
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (valid[i]) { psum[c] += v[i][c]; pmax[c] = fmaxf(pmax[c], v[i][c]); }
+      amax = fmaxf(amax, fabsf(v[i][c]));
+    }
+  }
+  // lanes sharing a channel group differ in the bits at and above log2(CPT)
+#pragma unroll
+  for (int o = CPT; o < 32; o <<= 1) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      psum[c] += __shfl_xor_sync(0xffffffffu, psum[c], o);
+      pmax[c] = fmaxf(pmax[c], __shfl_xor_sync(0xffffffffu, pmax[c], o));
+    }
+  }
+  __shared__ float s_sum[kThreads / 32][D];
+  __shared__ float s_max[kThreads / 32][D];
+  __shared__ float s_amax[kThreads / 32];
+  if (lane < CPT) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      s_sum[warp][cg * 8 + c] = psum[c];
+      s_max[warp][cg * 8 + c] = pmax[c];
+    }
+  }
+  amax = warp_max(amax);
+  if (lane == 0) s_amax[warp] = amax;
+  __syncthreads();
+  const size_t blk_lin = (size_t)bh * g.nb + blk;
+  if (tid < D) {
+    float s = 0.f, m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) { s += s_sum[w][tid]; m = fmaxf(m, s_max[w][tid]); }
+    P.avg[which][blk_lin * D + tid] = s / (float)block_real_count(g, blk);
+    P.mx[which][blk_lin * D + tid] = m;
+  }
+  amax = s_amax[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, s_amax[w]);
+
+  // ---- INT8: one symmetric scale per block
+  if (want_i8) {
+    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+    if (tid == 0) P.s8[which][blk_lin] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+    int8_t* __restrict__ dst = P.i8[which] + blk_lin * 64 * D;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const int s = slot0 + i * SLOT_STEP;
+      uint2 w;
+      w.x = quant_i8x4(v[i], inv);
+      w.y = quant_i8x4(v[i] + 4, inv);
+      *reinterpret_cast<uint2*>(dst + (size_t)s * D + cg * 8) = w;
+    }
+  }
+  // ---- NVFP4: e4m3 scale per 16 channels of a token
+  if (want_f4) {
+    uint8_t* __restrict__ dst = P.f4[which] + blk_lin * 64 * (D / 2);
+    uint8_t* __restrict__ sfd = P.sf4[which] + blk_lin * 64 * (D / 16);
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const int s = slot0 + i * SLOT_STEP;
+      float a8 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) a8 = fmaxf(a8, fabsf(v[i][c]));
+      const float a16 = fmaxf(a8, __shfl_xor_sync(0xffffffffu, a8, 1));
+      uint32_t sfb;
+      const uint32_t codes = quant_f4x8(v[i], a16, &sfb);
+      *reinterpret_cast<uint32_t*>(dst + (size_t)s * (D / 2) + cg * 4) = codes;
+      if ((cg & 1) == 0) sfd[(size_t)s * (D / 16) + cg / 2] = (uint8_t)sfb;
+    }
+  }
+}
+
+// Per-channel absmax of V over all real tokens of one head.
+template <int D>
+__global__ void __launch_bounds__(kThreads) v_amax_kernel(Geom g, const __nv_bfloat16* __restrict__ v,
+                                                          unsigned int* __restrict__ amax_bits,
+                                                          int tokens_per_cta) {
+  constexpr int CPT = D / 8;
+  constexpr int ROWS = kThreads / CPT;
+  const int bh = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid % CPT;
+  const int t0 = blockIdx.x * tokens_per_cta;
+  const int t1 = min(g.N, t0 + tokens_per_cta);
+  const __nv_bfloat16* __restrict__ x = v + (size_t)bh * g.N * D;
+  float m[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m[c] = 0.f;
+  for (int t = t0 + tid / CPT; t < t1; t += ROWS) {
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(x + (size_t)t * D + cg * 8), f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], fabsf(f[c]));
+  }
+#pragma unroll
+  for (int o = CPT; o < 32; o <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xffffffffu, m[c], o));
+  __shared__ float s_m[kThreads / 32][D];
+  if (lane < CPT)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) s_m[warp][cg * 8 + c] = m[c];
+  __syncthreads();
+  if (tid < D) {
+    float r = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) r = fmaxf(r, s_m[w][tid]);
+    atomicMax(amax_bits + (size_t)bh * D + tid, __float_as_uint(r));  // r >= 0: bit order = value order
+  }
+}
+
+struct VPtrs {
+  const __nv_bfloat16* v;
+  const unsigned int* amax_bits;
+  int8_t* i8;
+  float* s8;
+  uint8_t* f4;
+  uint8_t* sf4;
+  float* g4;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) pack_v_kernel(Geom g, VPtrs P, int want_i8, int want_f4) {
+  constexpr int CPT = D / 8;
+  constexpr int NC = 64 * CPT / kThreads;
+  constexpr int SLOT_STEP = kThreads / CPT;
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int cg = tid % CPT, slot0 = tid / CPT;
+  __shared__ float s_v[D][65];  // transposed tile [channel][slot], +1 against bank conflicts
+  const __nv_bfloat16* __restrict__ x = P.v + (size_t)bh * g.N * D;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int s = slot0 + i * SLOT_STEP;
+    const int tok = slot_token(g, blk, s);
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (tok >= 0) u = *reinterpret_cast<const uint4*>(x + (size_t)tok * D + cg * 8);
+    float f[8];
+    unpack8(u, f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) s_v[cg * 8 + c][s] = f[c];
+  }
+  __syncthreads();
+  const size_t blk_lin = (size_t)bh * g.nb + blk;
+  const unsigned int* amax_bits = P.amax_bits + (size_t)bh * D;
+  if (blk == 0 && tid < D) {
+    const float a = __uint_as_float(amax_bits[tid]);
+    if (want_i8) P.s8[(size_t)bh * D + tid] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
+    if (want_f4) P.g4[(size_t)bh * D + tid] = __fdiv_rn(a, 2688.0f);
+  }
+  // items: (channel c, 16-slot group j); 4 groups per channel
+  for (int item = tid; item < D * 4; item += kThreads) {
+    const int c = item >> 2, j = item & 3;
+    const float a = __uint_as_float(amax_bits[c]);
+    float f[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f[e] = s_v[c][16 * j + e];
+    if (want_i8) {
+      const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
+      uint4 w;
+      w.x = quant_i8x4(f, inv);
+      w.y = quant_i8x4(f + 4, inv);
+      w.z = quant_i8x4(f + 8, inv);
+      w.w = quant_i8x4(f + 12, inv);
+      *reinterpret_cast<uint4*>(P.i8 + (blk_lin * D + c) * 64 + 16 * j) = w;
+    }
+    if (want_f4) {
+      const float gch = __fdiv_rn(a, 2688.0f);
+      const float r = gch > 0.f ? __fdiv_rn(1.0f, gch) : 0.f;
+      float a16 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) { f[e] = __fmul_rn(f[e], r); a16 = fmaxf(a16, fabsf(f[e])); }
+      uint32_t sfb;
+      uint2 w;
+      w.x = quant_f4x8(f, a16, &sfb);
+      w.y = quant_f4x8(f + 8, a16, &sfb);
+      *reinterpret_cast<uint2*>(P.f4 + (blk_lin * D + c) * 32 + 8 * j) = w;
+      P.sf4[(blk_lin * D + c) * 4 + j] = (uint8_t)sfb;
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_prepare_d(const Geom& g, const Layout& L, const void* q, const void* k,
+                             const void* v, void* ws, cudaStream_t st) {
+  const int want_i8 = g.n8 > 0, want_f4 = g.n4 > 0;
+  PrepPtrs P;
+  P.x[0] = static_cast<const __nv_bfloat16*>(q);
+  P.x[1] = static_cast<const __nv_bfloat16*>(k);
+  P.avg[0] = at<float>(ws, L, R_Q_AVG); P.avg[1] = at<float>(ws, L, R_K_AVG);
+  P.mx[0] = at<float>(ws, L, R_Q_MAX); P.mx[1] = at<float>(ws, L, R_K_MAX);
+  P.i8[0] = at<int8_t>(ws, L, R_Q_I8); P.i8[1] = at<int8_t>(ws, L, R_K_I8);
+  P.s8[0] = at<float>(ws, L, R_Q_S8); P.s8[1] = at<float>(ws, L, R_K_S8);
+  P.f4[0] = at<uint8_t>(ws, L, R_Q_F4); P.f4[1] = at<uint8_t>(ws, L, R_K_F4);
+  P.sf4[0] = at<uint8_t>(ws, L, R_Q_SF4); P.sf4[1] = at<uint8_t>(ws, L, R_K_SF4);
+  P.perm = at<int>(ws, L, R_PERM);
+  prep_qk_kernel<D><<<dim3(g.nb, g.BH, 2), kThreads, 0, st>>>(g, P, want_i8, want_f4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !(want_i8 || want_f4)) return e;
+
+  unsigned int* amax = at<unsigned int>(ws, L, R_V_AMAX);
+  e = cudaMemsetAsync(amax, 0, L.size[R_V_AMAX], st);
+  if (e != cudaSuccess) return e;
+  const int tpc = 2048;
+  v_amax_kernel<D><<<dim3((g.N + tpc - 1) / tpc, g.BH), kThreads, 0, st>>>(
+      g, static_cast<const __nv_bfloat16*>(v), amax, tpc);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  VPtrs V{static_cast<const __nv_bfloat16*>(v), amax, at<int8_t>(ws, L, R_V_I8),
+          at<float>(ws, L, R_V_S8), at<uint8_t>(ws, L, R_V_F4), at<uint8_t>(ws, L, R_V_SF4),
+          at<float>(ws, L, R_V_G4)};
+  pack_v_kernel<D><<<dim3(g.nb, g.BH), kThreads, 0, st>>>(g, V, want_i8, want_f4);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prepare(const Geom& g, const Layout& L, const void* q, const void* k,
+                           const void* v, void* ws, cudaStream_t st) {
+  return g.d == 128 ? launch_prepare_d<128>(g, L, q, k, v, ws, st)
+                    : launch_prepare_d<64>(g, L, q, k, v, ws, st);
+}
+
+}  // namespace da2
