@@ -150,6 +150,34 @@ enum {
 };
 int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes);
 
+/* Allocation-free ranking.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory at call time — for
+ * example a host runtime that hands every byte of the GPU to its own arena at
+ * start-up, or a plugin hook invoked from another engine's execution path
+ * where allocating is not permitted — and so cannot provide the workspace
+ * that da2_rank_from_scores needs for its radix-select histograms.
+ *
+ * It computes exactly what da2_rank_from_scores computes (ranking and
+ * precision assignment of caller-given fp32 scores [B,H,nb,nb]) and writes the
+ * results to caller-given device buffers with the layouts of the MAP, LISTS
+ * and COUNTS workspace views: map uint8 [B,H,nb,nb], lists uint16 [B,H,nb,nb]
+ * (only the first c16+c8+c4 entries of a row are written), counts int32
+ * [B,H,nb,4].  All pointers are device pointers, 16-byte aligned.
+ *
+ * Scratch: a fixed array inside the library, sized for at most
+ * DA2_NOALLOC_MAX_HEADS (batch x head) pairs; larger problems return
+ * DA2_ERR_UNSUPPORTED before any device work.  Every GPU that loads the
+ * library keeps that array (about 1.5 MB) until the process exits.  The first
+ * call on a device looks the array's device address up (a runtime call); make
+ * that first call before any stream capture.  Calls on one device share the
+ * array: calls that may overlap on the GPU (different streams, no ordering)
+ * race and give wrong results; serialise them.  No call depends on what an
+ * earlier call left in the array.  The call allocates nothing: no cudaMalloc,
+ * no cudaFree, no allocating library routine. */
+#define DA2_NOALLOC_MAX_HEADS 64
+int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, uint16_t* lists,
+                     int32_t* counts, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* da2_status_string(int status);
 

@@ -169,6 +169,17 @@ int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t
   return DA2_OK;
 }
 
+int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, uint16_t* lists,
+                     int32_t* counts, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (g.BH > DA2_NOALLOC_MAX_HEADS) return DA2_ERR_UNSUPPORTED;
+  if (!aligned16(scores) || !aligned16(map) || !aligned16(lists) || !aligned16(counts)) return DA2_ERR_ARG;
+  if ((rc = check_device())) return rc;
+  return cuda_status(launch_rank_noalloc(g, scores, map, lists, counts, (cudaStream_t)stream));
+}
+
 const char* da2_status_string(int s) {
   switch (s) {
     case DA2_OK: return "ok";

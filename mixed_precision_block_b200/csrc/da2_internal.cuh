@@ -162,4 +162,6 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
                              const void* v, void* ws, void* out, cudaStream_t st);
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k,
                          const void* v, void* out, cudaStream_t st);
+cudaError_t launch_rank_noalloc(const Geom& g, const float* scores, uint8_t* map, uint16_t* lists,
+                                int* counts, cudaStream_t st);
 }  // namespace da2

@@ -16,6 +16,8 @@
 //                soon as its rank is the last one in its bucket
 // rank_assign    one CTA per query region: precision per pair, the u8 map and
 //                the per-query-block key lists (ballot/popc compaction)
+#include <mutex>
+
 #include "da2_internal.cuh"
 
 namespace da2 {
@@ -350,6 +352,72 @@ cudaError_t launch_rank(const Geom& g, const Layout& L, void* ws, bool hist0_don
   rank_assign_kernel<<<dim3(g.nb, g.BH), 256, 0, st>>>(g, scores, rs, at<uint8_t>(ws, L, R_MAP),
                                                        at<uint16_t>(ws, L, R_LISTS),
                                                        at<int>(ws, L, R_COUNTS));
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free ranking (da2_rank_noalloc).
+//
+// Same kernels and launch order as launch_rank on caller-given scores, but the
+// radix-select scratch (per-pass histograms and per-cut state) lives in this
+// file-scope device array instead of a caller workspace, so the call needs no
+// device allocation by anyone.  Every GPU that loads the library holds the
+// array (DA2_NOALLOC_MAX_HEADS heads' worth, about 1.5 MB) until the process
+// exits.  All calls on a device share it, so calls that overlap on the GPU
+// race; the histograms are cleared at the start of every call and the state is
+// rewritten by rank_init_kernel, so a call never depends on the previous one.
+constexpr size_t kNoallocHistBytes =
+    (size_t)kRankPasses * DA2_NOALLOC_MAX_HEADS * kTargets * 256 * sizeof(unsigned int);
+constexpr size_t kNoallocBytes =
+    kNoallocHistBytes + (size_t)DA2_NOALLOC_MAX_HEADS * kTargets * sizeof(RankState);
+static __device__ __align__(256) unsigned char g_rank_scratch[kNoallocBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64];  // device address of g_rank_scratch, per device ordinal
+
+// In host code `g_rank_scratch` names a host-side shadow, not device memory:
+// the device address has to be looked up once per device, with that device
+// current, before a kernel can be given it.
+cudaError_t rank_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_rank_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_rank_noalloc(const Geom& g, const float* scores, uint8_t* map, uint16_t* lists,
+                                int* counts, cudaStream_t st) {
+  if (g.BH > DA2_NOALLOC_MAX_HEADS) return cudaErrorInvalidValue;
+  void* base = nullptr;
+  cudaError_t e = rank_scratch_address(&base);
+  if (e != cudaSuccess) return e;
+  unsigned int* hist = static_cast<unsigned int*>(base);
+  RankState* rs = reinterpret_cast<RankState*>(static_cast<char*>(base) + kNoallocHistBytes);
+  const size_t used_hist = (size_t)kRankPasses * g.BH * kTargets * 256 * sizeof(unsigned int);
+  if ((e = cudaMemsetAsync(hist, 0, used_hist, st)) != cudaSuccess) return e;
+  const long long P = (long long)g.nb * g.nb;
+  const int per_cta = 16384;
+  const int nchunk = (int)((P + per_cta - 1) / per_cta);
+  rank_init_kernel<<<g.BH, 32, 0, st>>>(g, rs);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int pass = 0; pass < kRankPasses; ++pass) {
+    rank_hist_kernel<<<dim3(nchunk, g.BH), 256, 0, st>>>(g, scores, rs, hist, pass, per_cta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    rank_select_kernel<<<g.BH, 32, 0, st>>>(g, rs, hist, pass, pass == 0 ? 1 : 0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  rank_assign_kernel<<<dim3(g.nb, g.BH), 256, 0, st>>>(g, scores, rs, map, lists, counts);
   return cudaGetLastError();
 }
 

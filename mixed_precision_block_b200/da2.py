@@ -26,7 +26,8 @@ VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_
          "Q_F4", "K_F4", "Q_SF4", "K_SF4", "V_I8", "V_S8", "V_F4", "V_SF4", "V_G4",
          "SCORES", "MAP", "LISTS", "COUNTS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
-           "da2_dense_attention", "da2_debug_view", "da2_status_string"]
+           "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_status_string"]
+NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
 
 
 class Problem(ctypes.Structure):
@@ -63,6 +64,7 @@ _lib.da2_rank_from_scores.argtypes = [_P, _vp, _vp, _sz, _vp]
 _lib.da2_attention.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.da2_dense_attention.argtypes = [ctypes.c_int] * 4 + [_vp] * 5
 _lib.da2_debug_view.argtypes = [_P, _vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]
+_lib.da2_rank_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
 _lib.da2_status_string.argtypes = [ctypes.c_int]
 _lib.da2_status_string.restype = ctypes.c_char_p
 for _f in EXPORTS[:-1]:
@@ -119,6 +121,15 @@ def da2_draft_rank(p, ws, stream=None):
 def da2_rank_from_scores(p, scores, ws, stream=None):
     _check("da2_rank_from_scores", _lib.da2_rank_from_scores(ctypes.byref(p), _ptr(scores), _ptr(ws),
                                                              ws.numel(), _stream(stream, ws)))
+
+
+def da2_rank_noalloc(p, scores, prec_map, lists, counts, stream=None):
+    """Ranking + assignment without a workspace, for callers that cannot
+    allocate device memory at call time; its scratch is a fixed array inside
+    the library (at most NOALLOC_MAX_HEADS batch x head pairs).  Outputs go to
+    the caller's uint8 map, int16/uint16 lists and int32 counts tensors."""
+    _check("da2_rank_noalloc", _lib.da2_rank_noalloc(ctypes.byref(p), _ptr(scores), _ptr(prec_map),
+                                                     _ptr(lists), _ptr(counts), _stream(stream, scores)))
 
 
 def da2_attention(p, q, k, v, ws, out, stream=None):
