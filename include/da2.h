@@ -138,14 +138,17 @@ int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k
  *   MAP    uint8 [B*H][nb][nb]  precision per pair: 16, 8, 4 or 0 (skip)
  *   LISTS  uint16 [B*H][nb][nb] per query block: its 16-bit key blocks, then
  *          its 8-bit, then its 4-bit ones, each ascending
- *   COUNTS int32 [B*H][nb][4]   lengths of the three lists, 0 */
+ *   COUNTS int32 [B*H][nb][4]   lengths of the three lists, 0
+ *   STATUS int32 [1]            0, or 1 after a tensor-core attention call whose
+ *                               bounded pipeline waits expired (its output is
+ *                               then invalid); reset by every da2_attention */
 enum {
   DA2_VIEW_PERM = 0,
   DA2_VIEW_Q_AVG, DA2_VIEW_K_AVG, DA2_VIEW_Q_MAX, DA2_VIEW_K_MAX,
   DA2_VIEW_Q_I8, DA2_VIEW_K_I8, DA2_VIEW_Q_S8, DA2_VIEW_K_S8,
   DA2_VIEW_Q_F4, DA2_VIEW_K_F4, DA2_VIEW_Q_SF4, DA2_VIEW_K_SF4,
   DA2_VIEW_V_I8, DA2_VIEW_V_S8, DA2_VIEW_V_F4, DA2_VIEW_V_SF4, DA2_VIEW_V_G4,
-  DA2_VIEW_SCORES, DA2_VIEW_MAP, DA2_VIEW_LISTS, DA2_VIEW_COUNTS,
+  DA2_VIEW_SCORES, DA2_VIEW_MAP, DA2_VIEW_LISTS, DA2_VIEW_COUNTS, DA2_VIEW_STATUS,
   DA2_VIEW_COUNT_
 };
 int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes);

@@ -161,7 +161,7 @@ int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t
   static const Region map[DA2_VIEW_COUNT_] = {
       R_PERM, R_Q_AVG, R_K_AVG, R_Q_MAX, R_K_MAX, R_Q_I8, R_K_I8, R_Q_S8, R_K_S8,
       R_Q_F4, R_K_F4, R_Q_SF4, R_K_SF4, R_V_I8, R_V_S8, R_V_F4, R_V_SF4, R_V_G4,
-      R_SCORES, R_MAP, R_LISTS, R_COUNTS};
+      R_SCORES, R_MAP, R_LISTS, R_COUNTS, R_STATUS};
   if (which < 0 || which >= DA2_VIEW_COUNT_) return DA2_ERR_ARG;
   const Layout L = make_layout(g);
   *ptr = static_cast<char*>(ws) + L.off[map[which]];

@@ -186,8 +186,11 @@ __device__ __forceinline__ void block16(uint32_t sQ, uint32_t sK, uint32_t sV, u
   qk_16bit<D, false>(sQ, sK, warp, lane, S);
   float mx0, mx1;
   scale_mask(S, sl2, vmask, tq, mx0, mx1);
-  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-  const float al0 = fast_exp2(m[0] - mn0), al1 = fast_exp2(m[1] - mn1);
+  // the reference is the running max rounded up to an integer exponent, so
+  // P's bf16 rounding is relative to a power of two and rescales are exact
+  const float mn0 = fmaxf(m[0], ceilf(mx0)), mn1 = fmaxf(m[1], ceilf(mx1));
+  const float al0 = m[0] == -INFINITY ? 0.f : ldexpf(1.0f, (int)(m[0] - mn0));
+  const float al1 = m[1] == -INFINITY ? 0.f : ldexpf(1.0f, (int)(m[1] - mn1));
   m[0] = mn0; m[1] = mn1;
   float s0 = 0.f, s1 = 0.f;
 #pragma unroll
@@ -572,6 +575,9 @@ cudaError_t launch_dense_d(int B, int H, int N, const void* q, const void* k, co
 
 cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, const void* k, const void* v,
                              void* ws, void* out, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L, R_STATUS), 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  if (attention_tc_supported(g)) return launch_attention_tc(g, L, q, k, v, ws, out, st);
   return g.d == 128 ? launch_attention_d<128>(g, L, q, k, v, ws, out, st)
                     : launch_attention_d<64>(g, L, q, k, v, ws, out, st);
 }

@@ -34,6 +34,7 @@ enum Region {
   R_V_I8, R_V_S8, R_V_F4, R_V_SF4, R_V_G4,
   R_SCORES, R_MAP, R_LISTS, R_COUNTS,
   R_V_AMAX, R_LOGB, R_HIST, R_RSTATE,
+  R_PLIST, R_PCNT,
   R_COUNT_
 };
 
@@ -76,6 +77,9 @@ inline Layout make_layout(const Geom& g) {
   L.size[R_LOGB] = bh * nb * nb * 4;
   L.size[R_HIST] = (size_t)kRankPasses * bh * kTargets * 256 * 4;
   L.size[R_RSTATE] = bh * kTargets * sizeof(RankState);
+  // merged key lists of query-block pairs (2p, 2p+1): at most 2*nb entries each
+  L.size[R_PLIST] = bh * ((nb + 1) / 2) * (2 * nb) * 4;
+  L.size[R_PCNT] = bh * ((nb + 1) / 2) * 4 * 4;
   size_t o = 0;
   for (int r = 0; r < R_COUNT_; ++r) {
     L.off[r] = o;
@@ -143,6 +147,13 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   return h2;
 }
 
+// 2^x on the SFU (MUFU.EX2), flushing denormal results to zero.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // fp32 → key whose unsigned order is the float order (-0 canonicalised to +0).
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   uint32_t u = __float_as_uint(f + 0.0f);
@@ -162,6 +173,10 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
                              const void* v, void* ws, void* out, cudaStream_t st);
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k,
                          const void* v, void* out, cudaStream_t st);
+cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st);
+bool attention_tc_supported(const Geom& g);
+cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, const void* k,
+                                const void* v, void* ws, void* out, cudaStream_t st);
 cudaError_t launch_rank_noalloc(const Geom& g, const float* scores, uint8_t* map, uint16_t* lists,
                                 int* counts, cudaStream_t st);
 }  // namespace da2

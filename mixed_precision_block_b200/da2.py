@@ -24,7 +24,7 @@ DA2_OK, DA2_ERR_ARG, DA2_ERR_UNSUPPORTED, DA2_ERR_WORKSPACE, DA2_ERR_CUDA = rang
 
 VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_S8",
          "Q_F4", "K_F4", "Q_SF4", "K_SF4", "V_I8", "V_S8", "V_F4", "V_SF4", "V_G4",
-         "SCORES", "MAP", "LISTS", "COUNTS"]
+         "SCORES", "MAP", "LISTS", "COUNTS", "STATUS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
            "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_status_string"]
 NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
@@ -172,6 +172,7 @@ def view(p, ws, which) -> torch.Tensor:
         "V_G4": (torch.float32, (BH, d)),
         "SCORES": (torch.float32, (BH, nb, nb)), "MAP": (torch.uint8, (BH, nb, nb)),
         "LISTS": (torch.int16, (BH, nb, nb)), "COUNTS": (torch.int32, (BH, nb, 4)),
+        "STATUS": (torch.int32, (64,)),
     }[which if isinstance(which, str) else VIEWS[which]]
     return raw.view(spec[0]).view(spec[1])
 

@@ -22,9 +22,13 @@ Readings adopted (the pages leave these open):
   exp(m_blk - m) when merged into the shared accumulator.
 * the softmax denominator l sums the unquantised exp(s - m) over every retained
   real key of every phase.
-* 16-bit phase, ``emulate`` mode: P = bf16(exp(s - m_run)) with m_run the running
-  maximum over the 16-bit blocks seen so far (parity unpinned: the rounding
-  order is the GPU's choice).  ``math`` mode keeps P exact.
+* 16-bit phase, ``emulate`` mode: P is rounded to bf16 relative to a power of
+  two, 2^r with r = ceil(m_run * log2 e) and m_run the running maximum over the
+  16-bit blocks seen so far (ascending key blocks).  Because bf16 rounding
+  commutes with scaling by powers of two, the rounded P is then the same for
+  any integer-exponent reference a kernel keeps, however lazily it raises it
+  (parity unpinned beyond that: the GPU's exponential).  ``math`` mode keeps P
+  exact.
 * ``emulate`` mode rounds the output to bf16; a query block with no retained
   key block outputs zeros.
 """
@@ -35,6 +39,8 @@ import numpy as np
 
 from . import formats as F
 from .rank import BIT4, BIT8, BIT16
+
+LOG2E = 1.4426950408889634
 
 
 def bf16_round(x):
@@ -89,9 +95,12 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
         s = np.where(valid[kb][None, :], s, -np.inf)
         m_new = np.maximum(st.m, _row_max(s))
         if mode == "emulate":
-            # P is rounded relative to the running max, like the accumulator
+            # P is rounded in bf16 relative to 2^ceil(m_run log2 e), then brought
+            # to the accumulator's units (exp(-m_run)) exactly
             p_den = _exp_rel(s, m_new)
-            p_num = bf16_round(p_den)
+            r = np.ceil(m_new * LOG2E)
+            shift = np.exp2(r - m_new * LOG2E)  # >= 1; exact fp64 scaling
+            p_num = bf16_round(p_den / shift[:, None]) * shift[:, None]
             alpha = np.where(np.isfinite(st.m), np.exp(st.m - np.where(np.isfinite(m_new), m_new, 0)), 0.0)
             st.l = st.l * alpha + p_den.sum(1)
             st.o = st.o * alpha[:, None] + p_num @ prep["v_blocks"][kb]

@@ -47,6 +47,7 @@ def _full_check(wl, heads=None, dense_ref=True):
         if dense_ref:
             dn = PT.dense_rows(qh, kh, vh, toks)
             outs.append(PT.rel_l2(got, dn))
+    assert int(da2.view(p, ws, "STATUS")[0]) == 0
     return outs
 
 
@@ -61,6 +62,13 @@ def test_ragged_padded_grid_d128():
 
 def test_ragged_padded_grid_d64_batch2():
     wl = Workload("ragged64", 2, 2, 2, 13, 11, 64, 0.25, (30.0, 30.0, 30.0, 10.0), seed=4)
+    _full_check(wl)
+
+
+def test_odd_block_count_padded_d128_tensor_core_path():
+    # 27 region blocks (odd: the last query-block pair has one member), padded
+    # in y and x, budget without a 4-bit share
+    wl = Workload("odd", 1, 2, 3, 20, 20, 128, 0.5, (50.0, 0.0, 30.0, 20.0), seed=9)
     _full_check(wl)
 
 

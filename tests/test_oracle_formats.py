@@ -118,3 +118,12 @@ def test_bf16_round_matches_torch():
 @pytest.mark.parametrize("v", [0.0, -0.0])
 def test_signed_zero_codes(v):
     assert F.e2m1_encode(F.e2m1_round(v)) == (8 if np.signbit(v) else 0)
+
+
+def test_bf16_rounding_commutes_with_powers_of_two():
+    # the 16-bit phase's P rounding relies on it: rounding relative to any
+    # integer-exponent reference gives the same value
+    rng = np.random.default_rng(4)
+    x = rng.random(20000) * np.exp(rng.uniform(-30, 0, 20000))
+    for k in (-8, -3, 1, 5, 8):
+        np.testing.assert_array_equal(bf16_round(x * 2.0 ** k), bf16_round(x) * 2.0 ** k)
