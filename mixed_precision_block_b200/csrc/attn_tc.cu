@@ -2,8 +2,9 @@
 //
 // DraftAttention2 abstract and reading note (Method overview bullet 4): one
 // kernel runs a phase per precision for each query block, sharing data
-// movement, softmax statistics and one output accumulator.  DraftAttention (v1)
-// abstract: the output is restored to the original token order.
+// movement, softmax statistics and one output accumulator, and rescaling by the
+// quantisation scales at phase boundaries.  DraftAttention (v1) abstract: the
+// output is restored to the original token order.
 //
 // Tile shape.  A precision is assigned per (query block, key block) pair of 64
 // tokens each, so a single query block gives an M = 64 MMA, which runs the
@@ -14,25 +15,28 @@
 // and the other half's P rows are zero; on the video workloads 74-80 % of the
 // computed rows are useful, against 50 % for M = 64.
 //
-// Per key block j (warp roles: 4 softmax warps own one TMEM lane / tile row
-// each; one TMA producer warp; one MMA warp):
-//   16-bit  S = Q·K^T (kind::f16, bf16, M128 N64, fp32 in TMEM, 2 buffers);
-//           softmax threads turn their row into P = exp2(s − m_ref) in bf16
-//           (m_ref an integer exponent raised lazily: O is rescaled in TMEM, by
-//           a power of two, only when the row max grows by more than 2^8) and
-//           write it K-major to shared memory;
-//           O += P·V (kind::f16, V read MN-major straight from the TMA tile).
-//   8-bit   S = Q8·K8^T (kind::i8, s32); P8 = round(255·exp(s − m_blk)) (u8);
-//           X = P8·V8^T (kind::i8 u8×s8, s32, 2 buffers); the softmax thread
-//           merges X into O in TMEM with exp(m_blk − m)/255 and the channel
-//           scales (the phase-boundary rescale of the pages).
+// Roles (10 warps): warps 0-7 softmax — warp w owns TMEM lanes 32(w&3).. (tile
+// rows) and half h = w>>2 of every key block (keys 32h..32h+31) and of the
+// channels (64h..64h+63); warp 8 issues TMA loads; warp 9 issues the MMAs from
+// a non-blocking scheduler that starts S of a block as soon as its buffers are
+// free, ahead of the P·V of the block before.
+//   16-bit  S = Q·K^T (kind::f16 bf16, M128 N64, fp32 TMEM, 2 buffers);
+//           P = exp2(s·log2e/√d − m_ref) rounded to bf16, m_ref an integer
+//           exponent raised lazily (O rescaled in TMEM by a power of two only
+//           when the row max grows by more than 2^8); P goes K-major to shared
+//           memory; O += P·V (kind::f16, V read MN-major from the TMA tile).
+//   8-bit   S = Q8·K8^T (kind::i8, s32); P8 = round(255·exp(s − m_blk)) as u8;
+//           X = P8·V8^T (kind::i8 u8×s8, s32, 2 buffers); each softmax warp
+//           folds its 64 channels of X into a register accumulator weighted by
+//           exp(m_blk − m8); the per-channel V scale is applied once, at the
+//           phase boundary, when the register accumulator joins O.
 //   4-bit   handled by the legacy kernel (not routed here yet).
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), INT8 codes as 2-D
 // boxes of the workspace.  The epilogue writes O through the same region box
 // with a TMA store, whose clipping drops the padding rows — the restore.
 // Every mbarrier wait is bounded; on expiry the CTA raises the workspace status
-// word and skips ahead to release its tensor memory.
+// word, skips the rest and releases its tensor memory.
 #include <cuda.h>
 
 #include <mutex>
@@ -46,33 +50,45 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 192;  // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
-constexpr int kStages = 3;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q16 = 0;         // [2 halves][128 rows][128 B], SW128
 constexpr uint32_t SM_Q8 = 32768;      // [128 rows][128 B], SW128
-constexpr uint32_t SM_STAGE = 49152;   // kStages x 32 KB: K at +0, V at +16384
-constexpr uint32_t STAGE_BYTES = 32768;
-constexpr uint32_t SM_P = SM_STAGE + kStages * STAGE_BYTES;  // 2 x 16 KB
-constexpr uint32_t SM_VS = SM_P + 2 * 16384;                 // 128 fp32 V scales
-constexpr uint32_t SM_BAR = SM_VS + 512;                     // mbarriers
-constexpr uint32_t SM_MISC = SM_BAR + 256;
+constexpr uint32_t SM_STAGE = 49152;   // kStages x 64 KB, one unit each (below)
+constexpr uint32_t STAGE_BYTES = 65536;
+// 16-bit unit (key blocks a, b): K_a h0 | K_b h0 | K_a h1 | K_b h1 (8 KB each, so
+// each channel half of [K_a; K_b] is one 128-row K-major operand), V_a, V_b (16 KB)
+// INT8 unit (one key block): K8 at +0 (8 KB), V8^T at +32768 (8 KB)
+constexpr uint32_t ST_V = 32768;
+constexpr uint32_t SM_P = SM_STAGE + kStages * STAGE_BYTES;  // P_a | P_b, 16 KB each
+constexpr uint32_t SM_VS = SM_P + 32768;                     // 128 fp32 V channel scales
+constexpr uint32_t SM_RED = SM_VS + 512;                     // row-statistics exchange, 4 KB
+constexpr uint32_t SM_BAR = SM_RED + 4096;                   // mbarriers
+constexpr uint32_t SM_MISC = SM_BAR + 512;
 constexpr uint32_t SM_TOTAL = SM_MISC + 64;
 constexpr uint32_t kSmemBytes = SM_TOTAL + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns
-constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 256;  // S: 2 x 64, X: 2 x 128
+// TMEM columns: O 0-127, S 2 x 128 at 128 (a 16-bit unit fills 128, an INT8
+// unit 64), X 128 at 384
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384;
 
 // mbarrier slots (8 bytes each)
 enum {
   B_Q16 = 0, B_Q8, B_KV_FULL, B_KV_EMPTY = B_KV_FULL + kStages, B_S_FULL = B_KV_EMPTY + kStages,
-  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 2, B_X_FULL = B_P_FREE + 2,
-  B_X_FREE = B_X_FULL + 2, B_DONE = B_X_FREE + 2, B_COUNT
+  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_X_FULL = B_P_FREE + 1,
+  B_X_FREE = B_X_FULL + 1, B_DONE = B_X_FREE + 1,
+  B_PAIR = B_DONE + 1,   // [4 quarters][2 parities]: the two warps of a row quarter
+  B_EPI = B_PAIR + 8,    // [4 quarters]: final exchange
+  B_COUNT = B_EPI + 4
 };
-static_assert(B_COUNT * 8 <= 256, "barrier area");
+static_assert(B_COUNT * 8 <= 512, "barrier area");
 
 struct TcArgs {
   const uint32_t* plist;  // [BH][npairs][2*nb]
@@ -86,9 +102,30 @@ struct TcArgs {
 
 __device__ __forceinline__ void raise_timeout(int* status) { atomicOr(status, 1); }
 
+// Exact int32 -> fp32 for |x| < 2^22 on the integer and FMA pipes (the I2F
+// conversion unit is a narrow pipe): 1.5*2^23 + x has x in its low mantissa bits.
+__device__ __forceinline__ float i2f_small(uint32_t x) {
+  return __int_as_float((int)x + 0x4B400000) - 12582912.0f;
+}
+// round-to-nearest-even of a value in [0, 2^22) to an integer in the low bits,
+// again through the mantissa of 1.5*2^23 (the add rounds ties to even)
+__device__ __forceinline__ uint32_t rne_small(float v) {
+  return (uint32_t)__float_as_int(v + 12582912.0f) & 0x3FFFFFu;
+}
+
 // Items: kb | inA << 16 | inB << 17 | kind << 18 (kind 0 = 16-bit, 1 = 8-bit).
 __device__ __forceinline__ int item_kb(uint32_t e) { return (int)(e & 0xffffu); }
 __device__ __forceinline__ int item_kind(uint32_t e) { return (int)((e >> 18) & 3u); }
+
+__device__ __forceinline__ unsigned long long key_mask(const Geom& g, int kb) {
+  const int rx = kb % g.nrx, ry = (kb / g.nrx) % g.nry;
+  const int vy = min(g.rh, g.Hh - ry * g.rh), vx = min(g.rw, g.Ww - rx * g.rw);
+  if (vy == g.rh && vx == g.rw) return ~0ull;
+  const unsigned long long rowbits = (vx >= 64) ? ~0ull : ((1ull << vx) - 1ull);
+  unsigned long long m = 0;
+  for (int i = 0; i < vy; ++i) m |= rowbits << (g.rw * i);
+  return m;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -110,23 +147,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 8);
 
+  // units: 16-bit items are taken two at a time (one N = 128 score MMA per
+  // unit), INT8 items one at a time
+  const int nu16 = (n16 + 1) / 2;
+  const int nu = nu16 + n8;
+  auto unit_items = [&](int u, int& i0, int& cnt) {
+    if (u < nu16) { i0 = 2 * u; cnt = min(2, n16 - 2 * u); }
+    else { i0 = n16 + (u - nu16); cnt = 1; }
+  };
+
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q16), 1);
     mbar_init(bar(B_Q8), 1);
     for (int s = 0; s < kStages; ++s) { mbar_init(bar(B_KV_FULL + s), 1); mbar_init(bar(B_KV_EMPTY + s), 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_S_FULL + b), 1);
-      mbar_init(bar(B_S_FREE + b), 4);
-      mbar_init(bar(B_P_FULL + b), 4);
-      mbar_init(bar(B_P_FREE + b), 1);
-      mbar_init(bar(B_X_FULL + b), 1);
-      mbar_init(bar(B_X_FREE + b), 4);
+      mbar_init(bar(B_S_FREE + b), kSoftmaxWarps);
     }
+    mbar_init(bar(B_P_FULL), kSoftmaxWarps);
+    mbar_init(bar(B_P_FREE), 1);
+    mbar_init(bar(B_X_FULL), 1);
+    mbar_init(bar(B_X_FREE), kSoftmaxWarps);
     mbar_init(bar(B_DONE), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(B_PAIR + i), 2);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(B_EPI + i), 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(s0 + SM_MISC, 512);
+  if (warp == kMmaWarp) tmem_alloc(s0 + SM_MISC, 512);
   if (threadIdx.x < kD) reinterpret_cast<float*>(smem + SM_VS)[threadIdx.x] = A.v_s8[(size_t)bh * kD + threadIdx.x];
   tc_fence_before();
   __syncthreads();
@@ -140,7 +188,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     cx = rx * g.rw; cy = ry * g.rh; cf = bh * g.T + t;
   };
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- TMA producer
     if (elect_one()) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
@@ -161,306 +209,378 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_2d(s0 + SM_Q8, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qa) * 64);
         if (qb >= 0) tma_load_2d(s0 + SM_Q8 + 8192, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qb) * 64);
       }
-      for (int j = 0; j < n; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(bar(B_KV_EMPTY + s), ((j / kStages) - 1) & 1)) {
+      for (int u = 0; u < nu; ++u) {
+        const int s = u % kStages;
+        if (u >= kStages && !mbar_wait(bar(B_KV_EMPTY + s), ((u / kStages) - 1) & 1)) {
           raise_timeout(A.status); *abort_flag = 1; break;
         }
-        const uint32_t e = items[j];
-        const int kb = item_kb(e);
+        if (*abort_flag) break;
+        int i0, cnt;
+        unit_items(u, i0, cnt);
         const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
-        if (item_kind(e) == 0) {
-          mbar_expect_tx(bar(B_KV_FULL + s), 32768u);
-          box(kb, cx, cy, cf);
-          tma_load_4d(st, &tmK, bar(B_KV_FULL + s), 0, cx, cy, cf);
-          tma_load_4d(st + 8192, &tmK, bar(B_KV_FULL + s), 64, cx, cy, cf);
-          tma_load_4d(st + 16384, &tmV, bar(B_KV_FULL + s), 0, cx, cy, cf);
-          tma_load_4d(st + 16384 + 8192, &tmV, bar(B_KV_FULL + s), 64, cx, cy, cf);
+        const uint32_t fb = bar(B_KV_FULL + s);
+        if (u < nu16) {
+          mbar_expect_tx(fb, 32768u * (uint32_t)cnt);
+          for (int t = 0; t < cnt; ++t) {
+            box(item_kb(items[i0 + t]), cx, cy, cf);
+            tma_load_4d(st + t * 8192, &tmK, fb, 0, cx, cy, cf);
+            tma_load_4d(st + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
+            tma_load_4d(st + ST_V + t * 16384, &tmV, fb, 0, cx, cy, cf);
+            tma_load_4d(st + ST_V + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
+          }
         } else {
-          mbar_expect_tx(bar(B_KV_FULL + s), 16384u);
-          tma_load_2d(st, &tmK8, bar(B_KV_FULL + s), 0, (bh * g.nb + kb) * 64);
-          tma_load_2d(st + 16384, &tmV8, bar(B_KV_FULL + s), 0, (bh * g.nb + kb) * kD);
+          const int kb = item_kb(items[i0]);
+          mbar_expect_tx(fb, 16384u);
+          tma_load_2d(st, &tmK8, fb, 0, (bh * g.nb + kb) * 64);
+          tma_load_2d(st + ST_V, &tmV8, fb, 0, (bh * g.nb + kb) * kD);
         }
       }
     }
-  } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA scheduler
     if (elect_one()) {
-      const uint32_t id16 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 64);
+      const uint32_t id16n128 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 128);
+      const uint32_t id16n64 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 64);
       const uint32_t idpv = idesc(kDF32, kFmtBF16, kFmtBF16, false, true, 128, 128);
       const uint32_t id8 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
       const uint32_t idx8 = idesc(kDS32, kFmtU8, kFmtS8, false, false, 128, 128);
       bool ok = true;
       if (n16 > 0) ok = ok && mbar_wait(bar(B_Q16), 0);
       if (n8 > 0) ok = ok && mbar_wait(bar(B_Q8), 0);
-      int x_uses = 0;
-      auto issue_pv = [&](int i) -> bool {
-        const uint32_t e = items[i];
-        const int b = i & 1, s = i % kStages;
-        if (!mbar_wait(bar(B_P_FULL + b), (i >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
-        const uint32_t pb = s0 + SM_P + b * 16384;
-        if (item_kind(e) == 0) {
+      int sn = 0, pn = 0, xu = 0;  // next unit for S, next unit for P·V, INT8 results issued
+      uint32_t idle = 0;
+      while (ok && pn < nu) {
+        bool progressed = false;
+        if (sn < nu) {
+          const int s = sn % kStages, b = sn & 1;
+          if (mbar_test(bar(B_KV_FULL + s), (sn / kStages) & 1) &&
+              (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
+            const uint32_t sd = tbase + TM_S + b * 128;
+            if (sn < nu16) {
+              int i0, cnt;
+              unit_items(sn, i0, cnt);
+              const uint32_t id = cnt == 2 ? id16n128 : id16n64;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tbase + TM_O, smem_desc(pb + kk * 32, 16, 1024, SW_128),
-                    smem_desc(st + 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
-        } else {
-          const int xb = x_uses & 1;
-          if (x_uses >= 2 && !mbar_wait(bar(B_X_FREE + xb), ((x_uses >> 1) - 1) & 1)) return false;
-          tc_fence_after();
-          const uint32_t xt = tbase + TM_X + xb * 128;
+              for (int k = 0; k < 8; ++k) {
+                const int h = k >> 2, kk = k & 3;
+                mma_f16(sd, smem_desc(s0 + SM_Q16 + h * 16384 + kk * 32, 16, 1024, SW_128),
+                        smem_desc(st + h * 16384 + kk * 32, 16, 1024, SW_128), id, k > 0 ? 1u : 0u);
+              }
+            } else {
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_i8(xt, smem_desc(pb + kk * 32, 16, 512, SW_64), smem_desc(st + 16384 + kk * 32, 16, 512, SW_64),
-                   idx8, kk > 0 ? 1u : 0u);
-          mma_commit(bar(B_X_FULL + xb));
-          ++x_uses;
-        }
-        mma_commit(bar(B_P_FREE + b));
-        mma_commit(bar(B_KV_EMPTY + s));
-        return true;
-      };
-      for (int j = 0; ok && j < n; ++j) {
-        const uint32_t e = items[j];
-        const int s = j % kStages, b = j & 1;
-        if (!mbar_wait(bar(B_KV_FULL + s), (j / kStages) & 1)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(bar(B_S_FREE + b), ((j >> 1) - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
-        const uint32_t sd = tbase + TM_S + b * 64;
-        if (item_kind(e) == 0) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int h = k >> 2, kk = k & 3;
-            mma_f16(sd, smem_desc(s0 + SM_Q16 + h * 16384 + kk * 32, 16, 1024, SW_128),
-                    smem_desc(st + h * 8192 + kk * 32, 16, 1024, SW_128), id16, k > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
+                       smem_desc(st + kk * 32, 16, 1024, SW_128), id8, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(B_S_FULL + b));
+            ++sn;
+            progressed = true;
           }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
-                   smem_desc(st + kk * 32, 16, 1024, SW_128), id8, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(B_S_FULL + b));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        if (pn < sn) {
+          const int s = pn % kStages;
+          const bool int8 = pn >= nu16;
+          if (mbar_test(bar(B_P_FULL), pn & 1) && (!int8 || xu < 1 || mbar_test(bar(B_X_FREE), (xu - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
+            const uint32_t pbuf = s0 + SM_P;
+            if (!int8) {
+              int i0, cnt;
+              unit_items(pn, i0, cnt);
+              for (int t = 0; t < cnt; ++t) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_f16(tbase + TM_O, smem_desc(pbuf + t * 16384 + kk * 32, 16, 1024, SW_128),
+                          smem_desc(st + ST_V + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                mma_i8(tbase + TM_X, smem_desc(pbuf + kk * 32, 16, 512, SW_64),
+                       smem_desc(st + ST_V + kk * 32, 16, 512, SW_64), idx8, kk > 0 ? 1u : 0u);
+              mma_commit(bar(B_X_FULL));
+              ++xu;
+            }
+            mma_commit(bar(B_P_FREE));
+            mma_commit(bar(B_KV_EMPTY + s));
+            ++pn;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle > (1u << 26) || *abort_flag) {
+          ok = false;
+        }
       }
-      if (ok && n > 0) ok = issue_pv(n - 1);
       mma_commit(bar(B_DONE));
       if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps 0-3
-    const int row = threadIdx.x;  // TMEM lane and tile row
+    // ---------------------------------------------------------------- softmax warps 0-7
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;  // TMEM lane and tile row
     const bool in_b = row >= 64;
     const int qrow_blk = in_b ? qb : qa;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = kLog2e * rsqrtf((float)kD);
     const float sq = (n8 > 0 && qrow_blk >= 0) ? A.q_s8[(size_t)bh * g.nb + qrow_blk] : 0.f;
     const float* vs = reinterpret_cast<const float*>(smem + SM_VS);
-    float m_ref = -INFINITY, l = 0.f;
+    float* red = reinterpret_cast<float*>(smem + SM_RED);  // [2][2][128]
+    const unsigned FULL = 0xffffffffu;
+    // the two warps of a row quarter exchange row statistics through shared
+    // memory, ordered by an mbarrier (bounded wait, unlike a named barrier)
+    auto pair_sync = [&](int idx, uint32_t parity) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(idx));
+      return __all_sync(FULL, mbar_wait(bar(idx), parity));
+    };
+    float m16 = -INFINITY, l16 = 0.f;  // 16-bit phase: O in TMEM, integer reference
+    float m8 = -INFINITY, l8 = 0.f;    // 8-bit phase: register accumulator
     bool ok = true;
-    {  // O starts at zero
+    {  // O starts at zero (this warp's 64 columns)
       uint32_t z[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) z[i] = 0u;
-#pragma unroll
-      for (int c = 0; c < 128; c += 32) tmem_st32(tbase + lane_off + TM_O + c, z);
+      tmem_st32(tbase + lane_off + TM_O + half * 64, z);
+      tmem_st32(tbase + lane_off + TM_O + half * 64 + 32, z);
       tmem_wait_st();
     }
-    int x_uses = 0;
-    // INT8 block results are merged one INT8 item late, so that X of item i is
-    // computed while the softmax of the next item runs.
+    for (int u = 0; ok && u < nu16; ++u) {
+      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      const int b = u & 1;
+      int i0, cnt;
+      unit_items(u, i0, cnt);
+      float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
+      const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
+      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+        // ---- 16-bit unit: this warp owns key block `half` of the unit
+        const bool present = half < cnt;
+        const uint32_t e = present ? items[i0 + half] : 0u;
+        const bool member = present && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
+        uint32_t sr[64];
+        if (present) {
+          tmem_ld32(sbase + half * 64, sr);
+          tmem_ld32(sbase + half * 64 + 32, sr + 32);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
+        float mx = -INFINITY;
+        if (member) {
+          const unsigned long long vm = key_mask(g, item_kb(e));
+          if (vm == ~0ull) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
+              mx = fmaxf(mx, __uint_as_float(sr[i]));
+            }
+          }
+        }
+        xch[half * 128 + row] = mx;
+        if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+        mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * sl2;  // unit row max, log2 units
+        // the P buffer and O are free once the P·V of unit u-1 completed
+        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        const bool row_live = mx != -INFINITY;  // the row is a member of some block of the unit
+        const bool need = row_live && (mx > m16 + kRescaleThreshold || m16 == -INFINITY);
+        const bool need_o = need && m16 != -INFINITY;
+        if (__any_sync(FULL, need_o)) {
+          const float a = need_o ? ldexpf(1.0f, (int)(m16 - ceilf(mx))) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < 64; c += 32) {
+            uint32_t orr[32];
+            tmem_ld32(tbase + lane_off + TM_O + half * 64 + c, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * a);
+            tmem_st32(tbase + lane_off + TM_O + half * 64 + c, orr);
+          }
+          tmem_wait_st();
+          l16 *= a;
+        }
+        if (need) m16 = ceilf(mx);
+        if (present) {
+          uint32_t pw[32];
+          if (member) {
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m16));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m16));
+              sum += p0 + p1;
+              __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+              pw[i] = *reinterpret_cast<uint32_t*>(&hb);
+            }
+            l16 += sum;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pw[i] = 0u;
+          }
+          uint8_t* pb = smem + SM_P + half * 16384;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(pb + row * 128 + ((c ^ (row & 7)) * 16)) =
+                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P_FULL));
+    }
+    // the INT8 register accumulator lives only through the 8-bit phase
+    float o8[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) o8[i] = 0.f;
+    int xu = 0;
     bool have_pend = false, pend_member = false;
     float pend_mb = 0.f, pend_lb = 0.f;
+    // fold the X of the pending INT8 item into the register accumulator
     auto merge_x = [&]() -> bool {
-      const int xb = x_uses & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_X_FULL + xb), (x_uses >> 1) & 1))) return false;
+      if (!__all_sync(FULL, mbar_wait(bar(B_X_FULL), xu & 1))) return false;
       tc_fence_after();
       if (pend_member) {
-        const float mn = fmaxf(m_ref, pend_mb);
-        const float ao = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mn);
-        const float ab = fast_exp2(pend_mb - mn);
-        const float f = ab * (1.0f / 255.0f);
-        l = l * ao + pend_lb * ab;
-        m_ref = mn;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t xr[32], orr[32];
-          tmem_ld32(tbase + lane_off + TM_X + xb * 128 + c, xr);
-          tmem_ld32(tbase + lane_off + TM_O + c, orr);
-          tmem_wait_ld();
+        uint32_t xr[64];
+        tmem_ld32(tbase + lane_off + TM_X + half * 64, xr);
+        tmem_ld32(tbase + lane_off + TM_X + half * 64 + 32, xr + 32);
+        tmem_wait_ld();
+        if (pend_mb > m8 + kRescaleThreshold || m8 == -INFINITY) {
+          const float nm = ceilf(pend_mb);
+          const float a = (m8 == -INFINITY) ? 0.f : ldexpf(1.0f, (int)(m8 - nm));
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float o = __uint_as_float(orr[i]) * ao + f * vs[c + i] * (float)(int)xr[i];
-            orr[i] = __float_as_uint(o);
-          }
-          tmem_st32(tbase + lane_off + TM_O + c, orr);
+          for (int i = 0; i < 64; ++i) o8[i] *= a;
+          l8 *= a;
+          m8 = nm;
         }
-        tmem_wait_st();
+        const float w = fast_exp2(pend_mb - m8);
+        const float f = w * (1.0f / 255.0f);
+        l8 += pend_lb * w;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) o8[i] = fmaf(f, i2f_small(xr[i]), o8[i]);  // |X| < 64*255*127 < 2^22
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_X_FREE + xb));
-      ++x_uses;
+      if (lane == 0) mbar_arrive(bar(B_X_FREE));
+      ++xu;
       have_pend = false;
       return true;
     };
 
-    for (int j = 0; ok && j < n; ++j) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-      const uint32_t e = items[j];
-      const int kb = item_kb(e), kind = item_kind(e);
-      const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + b), (j >> 1) & 1))) { ok = false; break; }
+    for (int u = nu16; ok && u < nu; ++u) {
+      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      const int b = u & 1;
+      int i0, cnt;
+      unit_items(u, i0, cnt);
+      float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
+      const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
+      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tbase + lane_off + TM_S + b * 64, sr);
-      tmem_ld32(tbase + lane_off + TM_S + b * 64 + 32, sr + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
-
-      // real-key mask of the key block
-      unsigned long long vmask;
-      {
-        const int rx = kb % g.nrx, ry = (kb / g.nrx) % g.nry;
-        const int vy = min(g.rh, g.Hh - ry * g.rh), vx = min(g.rw, g.Ww - rx * g.rw);
-        const unsigned long long rowbits = (vx >= 64) ? ~0ull : ((1ull << vx) - 1ull);
-        vmask = 0;
-        for (int i = 0; i < vy; ++i) vmask |= rowbits << (g.rw * i);
-      }
-      float mb = -INFINITY, lb = 0.f;
-      uint32_t pw[32];  // packed P row: 32 x bf16x2 (16-bit) or 16 x u8x4 (8-bit)
-      if (kind == 0) {
+        // ---- INT8 unit: one key block; this warp owns keys 32*half..+31
+        const uint32_t e = items[i0];
+        const int kb = item_kb(e);
+        const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
+        uint32_t sr[32];
+        tmem_ld32(sbase + half * 32, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
+        const unsigned long long vm = key_mask(g, kb) >> (32 * half);
+        const bool full = (uint32_t)vm == 0xffffffffu;
+        int imx = INT_MIN;
         if (member) {
-          float mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float v = ((vmask >> i) & 1ull) ? __uint_as_float(sr[i]) * sl2 : -INFINITY;
-            sr[i] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
-          }
-          // raise the reference lazily; the O rescale is warp-collective (TMEM
-          // access), so a warp rescales when any of its rows needs it
-          const bool need = mx > m_ref + kRescaleThreshold || m_ref == -INFINITY;
-          const bool need_o = need && m_ref != -INFINITY;
-          if (__any_sync(0xffffffffu, need_o)) {
-            bool w_ok = j < 1 || mbar_wait(bar(B_P_FREE + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
-            if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-            tc_fence_after();
-            // the reference is an integer exponent, so the factor is a power of two
-            const float a = need_o ? ldexpf(1.0f, (int)(m_ref - ceilf(mx))) : 1.0f;
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 32) {
-              uint32_t orr[32];
-              tmem_ld32(tbase + lane_off + TM_O + c, orr);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * a);
-              tmem_st32(tbase + lane_off + TM_O + c, orr);
-            }
-            tmem_wait_st();
-            l *= a;
-          }
-          // P is exp2(s - m_ref) with m_ref = an integer >= max - 8: its bf16
-          // rounding is the same as relative to 2^ceil(row max), whatever the
-          // reference, since bf16 rounding commutes with powers of two
-          if (need) m_ref = ceilf(mx);
-          float sum = 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = fast_exp2(__uint_as_float(sr[2 * i]) - m_ref);
-            const float p1 = fast_exp2(__uint_as_float(sr[2 * i + 1]) - m_ref);
-            sum += p0 + p1;
-            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-            pw[i] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          l += sum;
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) pw[i] = 0u;
+          for (int i = 0; i < 32; ++i)
+            if (full || ((vm >> i) & 1ull)) imx = max(imx, (int)sr[i]);
         }
-      } else {
+        reinterpret_cast<int*>(xch)[half * 128 + row] = imx;
+        if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+        imx = max(imx, reinterpret_cast<const int*>(xch)[(1 - half) * 128 + row]);
+        float mb = -INFINITY, lb = 0.f;
+        uint32_t pw[8];
         if (member) {
           const float sc = sq * A.k_s8[(size_t)bh * g.nb + kb] * sl2;
+          mb = i2f_small((uint32_t)imx) * sc;  // sc >= 0: the max of the scores; |S| < 128*127^2 < 2^22
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float v = ((vmask >> i) & 1ull) ? (float)(int)sr[i] * sc : -INFINITY;
-            sr[i] = __float_as_uint(v);
-            mb = fmaxf(mb, v);
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             uint32_t w = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float p = fast_exp2(__uint_as_float(sr[4 * i + q]) - mb);
+              const int k = 4 * i + q;
+              float p = fast_exp2(fmaf(i2f_small(sr[k]), sc, -mb));
+              if (!full && !((vm >> k) & 1ull)) p = 0.f;
               lb += p;
-              w |= (__float2uint_rn(255.f * p) & 0xffu) << (8 * q);
+              w |= rne_small(255.f * p) << (8 * q);  // 255 p in [0, 255]
             }
             pw[i] = w;
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pw[i] = 0u;
+          for (int i = 0; i < 8; ++i) pw[i] = 0u;
         }
-      }
-      // P buffer b is free once the P·V of item j-2 completed
-      if (!__all_sync(0xffffffffu, j < 2 || mbar_wait(bar(B_P_FREE + b), ((j >> 1) - 1) & 1))) { ok = false; break; }
-      uint8_t* pb = smem + SM_P + b * 16384;
-      if (kind == 0) {
+        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        uint8_t* pb = smem + SM_P;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(pb + row * 128 + ((c ^ (row & 7)) * 16)) =
+        for (int c = 0; c < 2; ++c) {
+          const int chunk = half * 2 + c;
+          *reinterpret_cast<uint4*>(pb + row * 64 + ((chunk ^ ((row >> 1) & 3)) * 16)) =
               make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(pb + row * 64 + ((c ^ ((row >> 1) & 3)) * 16)) =
-              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL + b));
-      if (kind == 1) {
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_P_FULL));
         if (have_pend && !merge_x()) { ok = false; break; }
         have_pend = true;
         pend_member = member;
         pend_mb = mb;
         pend_lb = lb;
-      }
     }
     if (ok && have_pend) ok = merge_x();
-    // wait for every MMA, then the epilogue
-    if (ok && !__all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0))) ok = false;
+    if (ok && !__all_sync(FULL, mbar_wait(bar(B_DONE), 0))) ok = false;
     tc_fence_after();
     if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
-    // O row / l → bf16 → shared tile (reusing Q16's area, same SW128 layout) → TMA store
+    // ---- phase boundary and epilogue: O = (2^(m16-m) O16 + 2^(m8-m) sv ⊙ o8) / l
     {
-      const float il = (l > 0.f) ? 1.0f / l : 0.f;
-      uint8_t* ot = smem + SM_Q16;
-#pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      // both halves of a row carry partial sums; exchange them
+      float* lx = red + 512;  // [2 halves][2 values][128 rows], past the item buffers
+      lx[(half * 2 + 0) * 128 + row] = l16;
+      lx[(half * 2 + 1) * 128 + row] = l8;
+      if (!pair_sync(B_EPI + quarter, 0)) { raise_timeout(A.status); *abort_flag = 1; }
+      const float l16t = l16 + lx[((1 - half) * 2 + 0) * 128 + row];
+      const float l8t = l8 + lx[((1 - half) * 2 + 1) * 128 + row];
+      const float mm = fmaxf(m16, m8);
+      const float a16 = m16 == -INFINITY ? 0.f : fast_exp2(m16 - mm);
+      const float a8 = m8 == -INFINITY ? 0.f : fast_exp2(m8 - mm);
+      const float lt = l16t * a16 + l8t * a8;
+      const float il = lt > 0.f ? 1.0f / lt : 0.f;
+      uint8_t* ot = smem + SM_Q16 + half * 16384;  // channel half = output sub-tile
+#pragma unroll
+      for (int c = 0; c < 64; c += 32) {
         uint32_t orr[32];
-        tmem_ld32(tbase + lane_off + TM_O + c, orr);
+        tmem_ld32(tbase + lane_off + TM_O + half * 64 + c, orr);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(orr[2 * i]) * il,
-                                                   __uint_as_float(orr[2 * i + 1]) * il);
-          w[i] = *reinterpret_cast<uint32_t*>(&h);
+          const int ch = half * 64 + c + 2 * i;
+          const float v0 = (a16 * __uint_as_float(orr[2 * i]) + a8 * vs[ch] * o8[c + 2 * i]) * il;
+          const float v1 = (a16 * __uint_as_float(orr[2 * i + 1]) + a8 * vs[ch + 1] * o8[c + 2 * i + 1]) * il;
+          __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
+          w[i] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        const int half = c >> 6, ch0 = (c & 63) >> 3;  // 16-byte chunk index within the half
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = ch0 + q;
-          *reinterpret_cast<uint4*>(ot + half * 16384 + row * 128 + ((chunk ^ (row & 7)) * 16)) =
+          const int chunk = (c >> 3) + q;
+          *reinterpret_cast<uint4*>(ot + row * 128 + ((chunk ^ (row & 7)) * 16)) =
               make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
@@ -488,7 +608,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     // every issued MMA has completed before the columns are released
     (void)__all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0));
     tmem_relinquish();
