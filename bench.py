@@ -342,7 +342,8 @@ def run_ours(args, wl):
             "stages_ms": {"prepare": stage[0], "draft_rank": stage[1], "attention": stage[2]},
             "dense_bf16": {"ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
                            "speedup_of_sparse_call": dense_ms / ms},
-            "roofline": {"bound": "tensor", "kernel": "attn_mp_kernel", "achieved": achieved,
+            "roofline": {"bound": "tensor", "kernel": ("attn_tc_kernel" if wl.d == 128 and info.n4 == 0
+                                                        else "attn_mp_kernel"), "achieved": achieved,
                          "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
                          "traffic": traffic,
                          "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "

@@ -60,13 +60,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q16 = 0;         // [2 halves][128 rows][128 B], SW128
 constexpr uint32_t SM_Q8 = 32768;      // [128 rows][128 B], SW128
-constexpr uint32_t SM_STAGE = 49152;   // kStages x 64 KB, one unit each (below)
-constexpr uint32_t STAGE_BYTES = 65536;
-// 16-bit unit (key blocks a, b): K_a h0 | K_b h0 | K_a h1 | K_b h1 (8 KB each, so
-// each channel half of [K_a; K_b] is one 128-row K-major operand), V_a, V_b (16 KB)
-// INT8 unit (one key block): K8 at +0 (8 KB), V8^T at +32768 (8 KB)
-constexpr uint32_t ST_V = 32768;
-constexpr uint32_t SM_P = SM_STAGE + kStages * STAGE_BYTES;  // P_a | P_b, 16 KB each
+constexpr uint32_t SM_K = 49152;       // K ring: kStages x 32 KB
+constexpr uint32_t SM_V = SM_K + kStages * 32768;            // V ring: kStages x 32 KB
+// 16-bit unit (key blocks a, b): K slot = K_a h0 | K_b h0 | K_a h1 | K_b h1 (8 KB
+// each, so each channel half of [K_a; K_b] is one 128-row K-major operand);
+// V slot = V_a | V_b (16 KB each).  INT8 unit (one key block): K8 (8 KB), V8^T (8 KB).
+constexpr uint32_t SM_P = SM_V + kStages * 32768;            // P_a | P_b, 16 KB each
 constexpr uint32_t SM_VS = SM_P + 32768;                     // 128 fp32 V channel scales
 constexpr uint32_t SM_RED = SM_VS + 512;                     // row-statistics exchange, 4 KB
 constexpr uint32_t SM_BAR = SM_RED + 4096;                   // mbarriers
@@ -81,7 +80,8 @@ constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384;
 
 // mbarrier slots (8 bytes each)
 enum {
-  B_Q16 = 0, B_Q8, B_KV_FULL, B_KV_EMPTY = B_KV_FULL + kStages, B_S_FULL = B_KV_EMPTY + kStages,
+  B_Q16 = 0, B_Q8, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
+  B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages,
   B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_X_FULL = B_P_FREE + 1,
   B_X_FREE = B_X_FULL + 1, B_DONE = B_X_FREE + 1,
   B_PAIR = B_DONE + 1,   // [4 quarters][2 parities]: the two warps of a row quarter
@@ -107,15 +107,50 @@ __device__ __forceinline__ void raise_timeout(int* status) { atomicOr(status, 1)
 __device__ __forceinline__ float i2f_small(uint32_t x) {
   return __int_as_float((int)x + 0x4B400000) - 12582912.0f;
 }
+// packed fp32x2 arithmetic (one FMA-pipe instruction for two lanes' values)
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// bytes 0 of four words -> one word (x0 in the low byte)
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  uint32_t lo, hi, r;
+  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(x0), "r"(x1));
+  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(x2), "r"(x3));
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
+  return r;
+}
 // round-to-nearest-even of a value in [0, 2^22) to an integer in the low bits,
 // again through the mantissa of 1.5*2^23 (the add rounds ties to even)
 __device__ __forceinline__ uint32_t rne_small(float v) {
   return (uint32_t)__float_as_int(v + 12582912.0f) & 0x3FFFFFu;
 }
 
-// Items: kb | inA << 16 | inB << 17 | kind << 18 (kind 0 = 16-bit, 1 = 8-bit).
+// Items: kb | inA << 16 | inB << 17 | kind << 18 (kind 0 = 16-bit, 1 = 8-bit)
+//        | full << 20 (the key block has no padding slot).
 __device__ __forceinline__ int item_kb(uint32_t e) { return (int)(e & 0xffffu); }
 __device__ __forceinline__ int item_kind(uint32_t e) { return (int)((e >> 18) & 3u); }
+
+__device__ __forceinline__ bool item_full(uint32_t e) { return (e >> 20) & 1u; }
 
 __device__ __forceinline__ unsigned long long key_mask(const Geom& g, int kb) {
   const int rx = kb % g.nrx, ry = (kb / g.nrx) % g.nry;
@@ -159,7 +194,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q16), 1);
     mbar_init(bar(B_Q8), 1);
-    for (int s = 0; s < kStages; ++s) { mbar_init(bar(B_KV_FULL + s), 1); mbar_init(bar(B_KV_EMPTY + s), 1); }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_K_FULL + s), 1); mbar_init(bar(B_K_EMPTY + s), 1);
+      mbar_init(bar(B_V_FULL + s), 1); mbar_init(bar(B_V_EMPTY + s), 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_S_FULL + b), 1);
       mbar_init(bar(B_S_FREE + b), kSoftmaxWarps);
@@ -209,30 +247,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_2d(s0 + SM_Q8, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qa) * 64);
         if (qb >= 0) tma_load_2d(s0 + SM_Q8 + 8192, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qb) * 64);
       }
-      for (int u = 0; u < nu; ++u) {
-        const int s = u % kStages;
-        if (u >= kStages && !mbar_wait(bar(B_KV_EMPTY + s), ((u / kStages) - 1) & 1)) {
-          raise_timeout(A.status); *abort_flag = 1; break;
-        }
-        if (*abort_flag) break;
-        int i0, cnt;
-        unit_items(u, i0, cnt);
-        const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
-        const uint32_t fb = bar(B_KV_FULL + s);
-        if (u < nu16) {
-          mbar_expect_tx(fb, 32768u * (uint32_t)cnt);
-          for (int t = 0; t < cnt; ++t) {
-            box(item_kb(items[i0 + t]), cx, cy, cf);
-            tma_load_4d(st + t * 8192, &tmK, fb, 0, cx, cy, cf);
-            tma_load_4d(st + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
-            tma_load_4d(st + ST_V + t * 16384, &tmV, fb, 0, cx, cy, cf);
-            tma_load_4d(st + ST_V + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
+      // K of a unit is needed first (scores) and released first; V waits for
+      // the P·V two units back.  Issue whichever ring has room, K first.
+      int kn = 0, vn = 0;
+      uint32_t idle = 0;
+      while (kn < nu || vn < nu) {
+        bool progressed = false;
+        if (kn < nu && (kn < kStages || mbar_test(bar(B_K_EMPTY + kn % kStages), ((kn / kStages) - 1) & 1))) {
+          int i0, cnt;
+          unit_items(kn, i0, cnt);
+          const uint32_t dst = s0 + SM_K + (kn % kStages) * 32768;
+          const uint32_t fb = bar(B_K_FULL + kn % kStages);
+          if (kn < nu16) {
+            mbar_expect_tx(fb, 16384u * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t) {
+              box(item_kb(items[i0 + t]), cx, cy, cf);
+              tma_load_4d(dst + t * 8192, &tmK, fb, 0, cx, cy, cf);
+              tma_load_4d(dst + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
+            }
+          } else {
+            mbar_expect_tx(fb, 8192u);
+            tma_load_2d(dst, &tmK8, fb, 0, (bh * g.nb + item_kb(items[i0])) * 64);
           }
-        } else {
-          const int kb = item_kb(items[i0]);
-          mbar_expect_tx(fb, 16384u);
-          tma_load_2d(st, &tmK8, fb, 0, (bh * g.nb + kb) * 64);
-          tma_load_2d(st + ST_V, &tmV8, fb, 0, (bh * g.nb + kb) * kD);
+          ++kn;
+          progressed = true;
+        }
+        if (vn < kn && (vn < kStages || mbar_test(bar(B_V_EMPTY + vn % kStages), ((vn / kStages) - 1) & 1))) {
+          int i0, cnt;
+          unit_items(vn, i0, cnt);
+          const uint32_t dst = s0 + SM_V + (vn % kStages) * 32768;
+          const uint32_t fb = bar(B_V_FULL + vn % kStages);
+          if (vn < nu16) {
+            mbar_expect_tx(fb, 16384u * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t) {
+              box(item_kb(items[i0 + t]), cx, cy, cf);
+              tma_load_4d(dst + t * 16384, &tmV, fb, 0, cx, cy, cf);
+              tma_load_4d(dst + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
+            }
+          } else {
+            mbar_expect_tx(fb, 8192u);
+            tma_load_2d(dst, &tmV8, fb, 0, (bh * g.nb + item_kb(items[i0])) * kD);
+          }
+          ++vn;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle > (1u << 26) || *abort_flag) {
+          raise_timeout(A.status); *abort_flag = 1;
+          break;
         }
       }
     }
@@ -253,10 +316,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         bool progressed = false;
         if (sn < nu) {
           const int s = sn % kStages, b = sn & 1;
-          if (mbar_test(bar(B_KV_FULL + s), (sn / kStages) & 1) &&
+          if (mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1) &&
               (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1))) {
             tc_fence_after();
-            const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
+            const uint32_t st = s0 + SM_K + s * 32768;
             const uint32_t sd = tbase + TM_S + b * 128;
             if (sn < nu16) {
               int i0, cnt;
@@ -275,6 +338,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                        smem_desc(st + kk * 32, 16, 1024, SW_128), id8, kk > 0 ? 1u : 0u);
             }
             mma_commit(bar(B_S_FULL + b));
+            mma_commit(bar(B_K_EMPTY + s));
             ++sn;
             progressed = true;
           }
@@ -282,9 +346,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (pn < sn) {
           const int s = pn % kStages;
           const bool int8 = pn >= nu16;
-          if (mbar_test(bar(B_P_FULL), pn & 1) && (!int8 || xu < 1 || mbar_test(bar(B_X_FREE), (xu - 1) & 1))) {
+          if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL), pn & 1) &&
+              (!int8 || xu < 1 || mbar_test(bar(B_X_FREE), (xu - 1) & 1))) {
             tc_fence_after();
-            const uint32_t st = s0 + SM_STAGE + s * STAGE_BYTES;
+            const uint32_t st = s0 + SM_V + s * 32768;
             const uint32_t pbuf = s0 + SM_P;
             if (!int8) {
               int i0, cnt;
@@ -293,18 +358,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                   mma_f16(tbase + TM_O, smem_desc(pbuf + t * 16384 + kk * 32, 16, 1024, SW_128),
-                          smem_desc(st + ST_V + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
+                          smem_desc(st + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
               }
             } else {
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk)
                 mma_i8(tbase + TM_X, smem_desc(pbuf + kk * 32, 16, 512, SW_64),
-                       smem_desc(st + ST_V + kk * 32, 16, 512, SW_64), idx8, kk > 0 ? 1u : 0u);
+                       smem_desc(st + kk * 32, 16, 512, SW_64), idx8, kk > 0 ? 1u : 0u);
               mma_commit(bar(B_X_FULL));
               ++xu;
             }
             mma_commit(bar(B_P_FREE));
-            mma_commit(bar(B_KV_EMPTY + s));
+            mma_commit(bar(B_V_EMPTY + s));
             ++pn;
             progressed = true;
           }
@@ -372,29 +437,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
         float mx = -INFINITY;
         if (member) {
-          const unsigned long long vm = key_mask(g, item_kb(e));
-          if (vm == ~0ull) {
+          if (!item_full(e)) {
+            const unsigned long long vm = key_mask(g, item_kb(e));
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int i = 0; i < 64; ++i)
               if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
-              mx = fmaxf(mx, __uint_as_float(sr[i]));
-            }
           }
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 64; i += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
+          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
         }
         xch[half * 128 + row] = mx;
         if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
         mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * sl2;  // unit row max, log2 units
-        // the P buffer and O are free once the P·V of unit u-1 completed
-        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
-        tc_fence_after();
         const bool row_live = mx != -INFINITY;  // the row is a member of some block of the unit
         const bool need = row_live && (mx > m16 + kRescaleThreshold || m16 == -INFINITY);
         const bool need_o = need && m16 != -INFINITY;
+        const float a = need_o ? ldexpf(1.0f, (int)(m16 - ceilf(mx))) : 1.0f;
+        if (need) m16 = ceilf(mx);
+        // P of this warp's block, ahead of the wait for the previous P·V
+        uint32_t pw[32];
+        if (member) {
+          const uint64_t sl2x2 = f2pack(sl2, sl2), negm = f2pack(-m16, -m16);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float x0, x1;
+            f2unpack(f2fma(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            acc[i & 3] = f2add(acc[i & 3], f2pack(p0, p1));
+            __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+            pw[i] = *reinterpret_cast<uint32_t*>(&hb);
+          }
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2unpack(f2add(acc[0], acc[1]), s0, s1);
+          f2unpack(f2add(acc[2], acc[3]), s2, s3);
+          (void)s4; (void)s5; (void)s6; (void)s7;
+          l16 = l16 * a + ((s0 + s1) + (s2 + s3));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pw[i] = 0u;
+          l16 *= a;
+        }
+        // the P buffer and O are free once the P·V of unit u-1 completed
+        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
         if (__any_sync(FULL, need_o)) {
-          const float a = need_o ? ldexpf(1.0f, (int)(m16 - ceilf(mx))) : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < 64; c += 32) {
             uint32_t orr[32];
@@ -405,26 +496,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tmem_st32(tbase + lane_off + TM_O + half * 64 + c, orr);
           }
           tmem_wait_st();
-          l16 *= a;
         }
-        if (need) m16 = ceilf(mx);
         if (present) {
-          uint32_t pw[32];
-          if (member) {
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m16));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m16));
-              sum += p0 + p1;
-              __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-              pw[i] = *reinterpret_cast<uint32_t*>(&hb);
-            }
-            l16 += sum;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) pw[i] = 0u;
-          }
           uint8_t* pb = smem + SM_P + half * 16384;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
@@ -463,8 +536,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float w = fast_exp2(pend_mb - m8);
         const float f = w * (1.0f / 255.0f);
         l8 += pend_lb * w;
+        const uint64_t fx2 = f2pack(f, f), kx2 = f2pack(-12582912.0f, -12582912.0f);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) o8[i] = fmaf(f, i2f_small(xr[i]), o8[i]);  // |X| < 64*255*127 < 2^22
+        for (int i = 0; i < 64; i += 2) {  // |X| < 64*255*127 < 2^22: exact through the mantissa
+          const uint64_t xf = f2add(f2pack(__int_as_float((int)xr[i] + 0x4B400000),
+                                           __int_as_float((int)xr[i + 1] + 0x4B400000)), kx2);
+          f2unpack(f2fma(fx2, xf, f2pack(o8[i], o8[i + 1])), o8[i], o8[i + 1]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -481,11 +559,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       unit_items(u, i0, cnt);
       float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
       const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
+      // ---- INT8 unit: one key block; this warp owns keys 32*half..+31
+      const uint32_t e = items[i0];
+      const int kb = item_kb(e);
+      const float sk = A.k_s8[(size_t)bh * g.nb + kb];  // issued before the wait
       if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
       tc_fence_after();
-        // ---- INT8 unit: one key block; this warp owns keys 32*half..+31
-        const uint32_t e = items[i0];
-        const int kb = item_kb(e);
         const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
         uint32_t sr[32];
         tmem_ld32(sbase + half * 32, sr);
@@ -493,13 +572,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
-        const unsigned long long vm = key_mask(g, kb) >> (32 * half);
+        const unsigned long long vm = item_full(e) ? ~0ull : (key_mask(g, kb) >> (32 * half));
         const bool full = (uint32_t)vm == 0xffffffffu;
         int imx = INT_MIN;
         if (member) {
+          if (!full) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (full || ((vm >> i) & 1ull)) imx = max(imx, (int)sr[i]);
+            for (int i = 0; i < 32; ++i)
+              if (!((vm >> i) & 1ull)) sr[i] = (uint32_t)INT_MIN;
+          }
+          int i4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) i4[i & 3] = max(i4[i & 3], (int)sr[i]);
+          imx = max(max(i4[0], i4[1]), max(i4[2], i4[3]));
         }
         reinterpret_cast<int*>(xch)[half * 128 + row] = imx;
         if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
@@ -507,21 +592,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         float mb = -INFINITY, lb = 0.f;
         uint32_t pw[8];
         if (member) {
-          const float sc = sq * A.k_s8[(size_t)bh * g.nb + kb] * sl2;
+          const float sc = sq * sk * sl2;
           mb = i2f_small((uint32_t)imx) * sc;  // sc >= 0: the max of the scores; |S| < 128*127^2 < 2^22
+          const uint64_t scx2 = f2pack(sc, sc), negm = f2pack(-mb, -mb);
+          const uint64_t kx2 = f2pack(-12582912.0f, -12582912.0f);
+          const uint64_t c255 = f2pack(255.0f, 255.0f), kmag = f2pack(12582912.0f, 12582912.0f);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            uint32_t w = 0;
+            uint32_t c[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 4; q += 2) {
               const int k = 4 * i + q;
-              float p = fast_exp2(fmaf(i2f_small(sr[k]), sc, -mb));
-              if (!full && !((vm >> k) & 1ull)) p = 0.f;
-              lb += p;
-              w |= rne_small(255.f * p) << (8 * q);  // 255 p in [0, 255]
+              // exact int -> float through the mantissa of 1.5*2^23, then the score
+              const uint64_t sf = f2add(f2pack(__int_as_float((int)sr[k] + 0x4B400000),
+                                               __int_as_float((int)sr[k + 1] + 0x4B400000)), kx2);
+              float x0, x1;
+              f2unpack(f2fma(sf, scx2, negm), x0, x1);
+              float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              if (!full) {  // padding keys contribute nothing, whatever the block scale
+                if (!((vm >> k) & 1ull)) p0 = 0.f;
+                if (!((vm >> (k + 1)) & 1ull)) p1 = 0.f;
+              }
+              const uint64_t pp = f2pack(p0, p1);
+              acc[(i * 2 + (q >> 1)) & 3] = f2add(acc[(i * 2 + (q >> 1)) & 3], pp);
+              float r0, r1;  // 255 p + 1.5*2^23: round-to-nearest-even code in the low byte
+              f2unpack(f2fma(pp, c255, kmag), r0, r1);
+              c[q] = __float_as_uint(r0);
+              c[q + 1] = __float_as_uint(r1);
             }
-            pw[i] = w;
+            pw[i] = pack_low_bytes(c[0], c[1], c[2], c[3]);
           }
+          float s0, s1, s2, s3;
+          f2unpack(f2add(acc[0], acc[1]), s0, s1);
+          f2unpack(f2add(acc[2], acc[3]), s2, s3);
+          lb = (s0 + s1) + (s2 + s3);
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) pw[i] = 0u;
@@ -624,7 +729,8 @@ namespace da2 {
 namespace {
 
 // Merged key lists of query-block pairs (2p, 2p+1): per phase (16, 8, 4) the
-// ascending key blocks either member keeps in that phase, with member flags.
+// ascending key blocks either member keeps in that phase, with member flags and
+// a flag for key blocks without padding.
 __global__ void __launch_bounds__(256) pair_lists_kernel(Geom g, const uint8_t* __restrict__ map,
                                                          uint32_t* __restrict__ plist, int* __restrict__ pcnt,
                                                          int npairs) {
@@ -654,7 +760,10 @@ __global__ void __launch_bounds__(256) pair_lists_kernel(Geom g, const uint8_t* 
         int off = run;
         for (int w = 0; w < warp; ++w) off += wtot[w];
         off += __popc(bal & ((1u << lane) - 1u));
-        out[off] = (uint32_t)kb | ((uint32_t)a << 16) | ((uint32_t)b << 17) | ((uint32_t)ph << 18);
+        const int rx = kb % g.nrx, ry = (kb / g.nrx) % g.nry;
+        const bool full = (ry + 1) * g.rh <= g.Hh && (rx + 1) * g.rw <= g.Ww;
+        out[off] = (uint32_t)kb | ((uint32_t)a << 16) | ((uint32_t)b << 17) | ((uint32_t)ph << 18) |
+                   ((uint32_t)full << 20);
       }
       for (int w = 0; w < 8; ++w) run += wtot[w];
       __syncthreads();
