@@ -130,10 +130,14 @@ int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k
  *   Q_AVG/K_AVG/Q_MAX/K_MAX  fp32 [B*H][nb][d]
  *   Q_I8/K_I8  int8 [B*H][nb][64][d];  Q_S8/K_S8 fp32 [B*H][nb]
  *   Q_F4/K_F4  uint8 [B*H][nb][64][d/2] (even channel in the low nibble)
- *   Q_SF4/K_SF4 uint8 e4m3 [B*H][nb][64][d/16]
+ *   Q_SF4/K_SF4 uint8 e4m3 [B*H][nb][d/64][32][16]: per 64-channel chunk an
+ *          atom whose line i holds the 4 scales (16 channels each) of slots i
+ *          and i+32 as two 32-bit words, repeated in words 2-3 (the layout the
+ *          tensor core reads scale factors from)
  *   V_I8  int8 [B*H][nb][d][64];  V_S8 fp32 [B*H][d]
  *   V_F4  uint8 [B*H][nb][d][32] (even token in the low nibble)
- *   V_SF4 uint8 e4m3 [B*H][nb][d][4];  V_G4 fp32 [B*H][d]
+ *   V_SF4 uint8 e4m3 [B*H][nb][32][16]: line i holds the 4 scales (16 tokens
+ *          each) of channels i, i+32, i+64, i+96;  V_G4 fp32 [B*H][d]
  *   SCORES fp32 [B*H][nb][nb]
  *   MAP    uint8 [B*H][nb][nb]  precision per pair: 16, 8, 4 or 0 (skip)
  *   LISTS  uint16 [B*H][nb][nb] per query block: its 16-bit key blocks, then

@@ -39,8 +39,9 @@ struct SmemLayout {
   static constexpr int K = Q + TILE16;       // 2 stages
   static constexpr int V = K + 2 * TILE16;   // 2 stages
   static constexpr int RAW = V + 2 * TILE16; // 2 stages of NVFP4 codes + scales
-  static constexpr int RAW_KC = 0, RAW_KS = 64 * D / 2, RAW_VC = RAW_KS + 64 * D / 16,
-                       RAW_VS = RAW_VC + D * 32, RAW_STAGE = RAW_VS + D * 4;
+  static constexpr int KSF = (D / 64) * kSfAtomBytes;  // K scales of one block
+  static constexpr int RAW_KC = 0, RAW_KS = 64 * D / 2, RAW_VC = RAW_KS + KSF,
+                       RAW_VS = RAW_VC + D * 32, RAW_STAGE = RAW_VS + kSfAtomBytes;
   static constexpr int P = RAW + 2 * RAW_STAGE;  // per warp [16][64] u8
   static constexpr int VS = P + kWarps * 1024;   // per-channel V scale (fp32)
   static constexpr int TOTAL = VS + D * 4;
@@ -97,7 +98,7 @@ __device__ __forceinline__ void load_bytes(uint32_t dst, const uint8_t* src, int
     cp_async16(dst + e * 16, src + e * 16, 16);
 }
 
-// Dequantise an NVFP4 tile (codes [rows][cols/2], e4m3 scales [rows][cols/16])
+// Dequantise an NVFP4 tile (codes [rows][cols/2], e4m3 scales in the atom layout)
 // to f16 [rows][cols] in a swizzled shared tile.  Every value e2m1 × e4m3 is
 // exact in f16.  `codes`/`scales` may be global or shared (generic pointers).
 template <int COLS>
@@ -107,7 +108,7 @@ __device__ __forceinline__ void dequant_f4_tile(uint8_t* dst, const uint8_t* cod
   for (int e = threadIdx.x; e < rows * CPR; e += kAttnThreads) {
     const int r = e / CPR, c = e % CPR;
     const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + (size_t)r * (COLS / 2) + c * 4);
-    const uint32_t sb = scales[(size_t)r * (COLS / 16) + c / 2];
+    const uint32_t sb = scales[sf_atom_offset(r, c / 2)];
     uint32_t h2;
     {
       const uint16_t b = (uint16_t)(sb | (sb << 8));
@@ -465,15 +466,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_mp_kernel(Geom g, AttnAr
   // ---------------- phase 4
   if (cnt.z > 0) {
     const uint16_t* l4 = list + cnt.x + cnt.y;
-    dequant_f4_tile<D>(smem + SL::Q, A.q_f4 + row_lin * 64 * (D / 2), A.q_sf4 + row_lin * 64 * (D / 16), 64);
+    dequant_f4_tile<D>(smem + SL::Q, A.q_f4 + row_lin * 64 * (D / 2), A.q_sf4 + row_lin * SL::KSF, 64);
     for (int c = threadIdx.x; c < D; c += kAttnThreads) vs[c] = A.v_g4[(size_t)bh * D + c];
     auto issue = [&](int j) {
       const size_t kl = (size_t)bh * g.nb + l4[j];
       const uint32_t raw = s0 + SL::RAW + (j & 1) * SL::RAW_STAGE;
       load_bytes(raw + SL::RAW_KC, A.k_f4 + kl * 64 * (D / 2), 64 * D / 2);
-      load_bytes(raw + SL::RAW_KS, A.k_sf4 + kl * 64 * (D / 16), 64 * D / 16);
+      load_bytes(raw + SL::RAW_KS, A.k_sf4 + kl * SL::KSF, SL::KSF);
       load_bytes(raw + SL::RAW_VC, A.v_f4 + kl * D * 32, D * 32);
-      load_bytes(raw + SL::RAW_VS, A.v_sf4 + kl * D * 4, D * 4);
+      load_bytes(raw + SL::RAW_VS, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes);
       cp_async_commit();
     };
     issue(0);

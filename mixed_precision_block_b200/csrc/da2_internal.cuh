@@ -15,6 +15,16 @@ constexpr int kBlockTokens = 64;     // one region = one 64-token block
 constexpr int kRankPasses = 8;       // 64-bit ranking key, 8 bits per pass
 constexpr int kTargets = 3;          // rank cuts: n16, n16+n8, n16+n8+n4
 
+// NVFP4 e4m3 scales are stored in the layout the tensor core reads them from
+// (tcgen05.cp 32x128b.warpx4): per 64-element chunk of the reduction axis, an
+// atom of 32 lines x 16 bytes in which line i holds the 4 scales (one per 16
+// elements) of rows i, i+32, i+64, i+96 as four 32-bit words.  A 64-row Q/K
+// block fills words 0 and 1 of each line and repeats them in words 2 and 3.
+constexpr int kSfAtomBytes = 512;
+__host__ __device__ __forceinline__ int sf_atom_offset(int row, int mb) {
+  return (mb >> 2) * kSfAtomBytes + (row & 31) * 16 + (row >> 5) * 4 + (mb & 3);
+}
+
 // Geometry of one problem, derived once on the host and passed by value.
 struct Geom {
   int B, H, T, Hh, Ww, d, rh, rw;
@@ -63,11 +73,11 @@ inline Layout make_layout(const Geom& g) {
   L.size[R_Q_I8] = L.size[R_K_I8] = bh * nb * S * d;
   L.size[R_Q_S8] = L.size[R_K_S8] = bh * nb * 4;
   L.size[R_Q_F4] = L.size[R_K_F4] = bh * nb * S * d / 2;
-  L.size[R_Q_SF4] = L.size[R_K_SF4] = bh * nb * S * d / 16;
+  L.size[R_Q_SF4] = L.size[R_K_SF4] = bh * nb * (d / 64) * kSfAtomBytes;
   L.size[R_V_I8] = bh * nb * d * S;
   L.size[R_V_S8] = bh * d * 4;
   L.size[R_V_F4] = bh * nb * d * S / 2;
-  L.size[R_V_SF4] = bh * nb * d * S / 16;
+  L.size[R_V_SF4] = bh * nb * kSfAtomBytes;
   L.size[R_V_G4] = bh * d * 4;
   L.size[R_SCORES] = bh * nb * nb * 4;
   L.size[R_MAP] = bh * nb * nb;

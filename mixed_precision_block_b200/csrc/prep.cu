@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads) prep_qk_kernel(Geom g, PrepPtrs P, i
   // ---- NVFP4: e4m3 scale per 16 channels of a token
   if (want_f4) {
     uint8_t* __restrict__ dst = P.f4[which] + blk_lin * 64 * (D / 2);
-    uint8_t* __restrict__ sfd = P.sf4[which] + blk_lin * 64 * (D / 16);
+    uint8_t* __restrict__ sfd = P.sf4[which] + blk_lin * (D / 64) * kSfAtomBytes;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
       const int s = slot0 + i * SLOT_STEP;
@@ -179,7 +179,11 @@ __global__ void __launch_bounds__(kThreads) prep_qk_kernel(Geom g, PrepPtrs P, i
       uint32_t sfb;
       const uint32_t codes = quant_f4x8(v[i], a16, &sfb);
       *reinterpret_cast<uint32_t*>(dst + (size_t)s * (D / 2) + cg * 4) = codes;
-      if ((cg & 1) == 0) sfd[(size_t)s * (D / 16) + cg / 2] = (uint8_t)sfb;
+      if ((cg & 1) == 0) {
+        const int o = sf_atom_offset(s, cg / 2);
+        sfd[o] = (uint8_t)sfb;
+        sfd[o + 8] = (uint8_t)sfb;  // rows 64..127 of the atom repeat rows 0..63
+      }
     }
   }
 }
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(kThreads) pack_v_kernel(Geom g, VPtrs P, int w
       w.x = quant_f4x8(f, a16, &sfb);
       w.y = quant_f4x8(f + 8, a16, &sfb);
       *reinterpret_cast<uint2*>(P.f4 + (blk_lin * D + c) * 32 + 8 * j) = w;
-      P.sf4[(blk_lin * D + c) * 4 + j] = (uint8_t)sfb;
+      P.sf4[blk_lin * kSfAtomBytes + sf_atom_offset(c, j)] = (uint8_t)sfb;
     }
   }
 }

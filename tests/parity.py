@@ -54,6 +54,28 @@ def unpack_nibbles(t):
     return out
 
 
+def qk_sf_natural(atoms):
+    """[nb, d/64, 32, 16] scale atoms -> [nb, 64, d/16] (slot, microblock); checks the repeat."""
+    a = np.asarray(atoms)
+    nb, nch = a.shape[0], a.shape[1]
+    words = a.reshape(nb, nch, 32, 4, 4)  # [blk, chunk, line, word, byte]
+    np.testing.assert_array_equal(words[:, :, :, 2:], words[:, :, :, :2])
+    out = np.empty((nb, 64, nch * 4), dtype=np.uint8)
+    for w in range(2):
+        for c in range(nch):
+            out[:, 32 * w:32 * w + 32, 4 * c:4 * c + 4] = words[:, c, :, w, :]
+    return out
+
+
+def v_sf_natural(atoms, d):
+    """[nb, 32, 16] scale atoms -> [nb, d, 4] (channel, microblock)."""
+    a = np.asarray(atoms).reshape(-1, 32, 4, 4)  # [blk, line, word, byte]
+    out = np.empty((a.shape[0], d, 4), dtype=np.uint8)
+    for w in range(d // 32):
+        out[:, 32 * w:32 * w + 32, :] = a[:, :, w, :]
+    return out
+
+
 def g(p, ws, name, bh=None):
     t = da2.view(p, ws, name)
     if bh is not None and name != "PERM":
@@ -81,14 +103,16 @@ def check_prep_head(p, ws, op, pr, bh, n8, n4, blocks=None):
         if n4:
             np.testing.assert_array_equal(unpack_nibbles(da2.view(p, ws, f"{T}_F4")[bh])[sel], pr[f"{t}_f4"][sel],
                                           err_msg=f"{T}_F4")
-            np.testing.assert_array_equal(g(p, ws, f"{T}_SF4", bh)[sel], pr[f"{t}_sf4"][sel], err_msg=f"{T}_SF4")
+            np.testing.assert_array_equal(qk_sf_natural(g(p, ws, f"{T}_SF4", bh))[sel], pr[f"{t}_sf4"][sel],
+                                          err_msg=f"{T}_SF4")
     if n8:
         np.testing.assert_array_equal(g(p, ws, "V_I8", bh)[sel], pr["v_i8"][sel], err_msg="V_I8")
         np.testing.assert_array_equal(g(p, ws, "V_S8", bh).astype(np.float64), pr["v_s8"])
     if n4:
         np.testing.assert_array_equal(unpack_nibbles(da2.view(p, ws, "V_F4")[bh])[sel], pr["v_f4"][sel],
                                       err_msg="V_F4")
-        np.testing.assert_array_equal(g(p, ws, "V_SF4", bh)[sel], pr["v_sf4"][sel], err_msg="V_SF4")
+        np.testing.assert_array_equal(v_sf_natural(g(p, ws, "V_SF4", bh), op.d)[sel], pr["v_sf4"][sel],
+                                      err_msg="V_SF4")
         np.testing.assert_array_equal(g(p, ws, "V_G4", bh).astype(np.float64), pr["v_g4"])
 
 
