@@ -30,7 +30,13 @@
 //           folds its 64 channels of X into a register accumulator weighted by
 //           exp(m_blk − m8); the per-channel V scale is applied once, at the
 //           phase boundary, when the register accumulator joins O.
-//   4-bit   handled by the legacy kernel (not routed here yet).
+//   4-bit   S = Q4·K4^T (kind::mxf4nvf4, block16 e4m3 scales copied into TMEM
+//           with tcgen05.cp from the scale atoms prep wrote); P re-quantised to
+//           NVFP4 per 16 keys in registers, with its scales written as an atom;
+//           X = P4·V4^T (block-scaled, fp32), folded into the register
+//           accumulator; the channel scale g is applied at the end.  Entering
+//           the phase, the INT8 accumulator is folded into O with its own
+//           channel scale first — the phase-boundary rescale.
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), INT8 codes as 2-D
 // boxes of the workspace.  The epilogue writes O through the same region box
@@ -66,21 +72,29 @@ constexpr uint32_t SM_V = SM_K + kStages * 32768;            // V ring: kStages 
 // each, so each channel half of [K_a; K_b] is one 128-row K-major operand);
 // V slot = V_a | V_b (16 KB each).  INT8 unit (one key block): K8 (8 KB), V8^T (8 KB).
 constexpr uint32_t SM_P = SM_V + kStages * 32768;            // P_a | P_b, 16 KB each
-constexpr uint32_t SM_VS = SM_P + 32768;                     // 128 fp32 V channel scales
-constexpr uint32_t SM_RED = SM_VS + 512;                     // row-statistics exchange, 4 KB
+constexpr uint32_t SM_VS = SM_P + 32768;                     // V channel scales: INT8 | NVFP4 g (fp32)
+constexpr uint32_t SM_RED = SM_VS + 1024;                    // row-statistics exchange, 4 KB
 constexpr uint32_t SM_BAR = SM_RED + 4096;                   // mbarriers
 constexpr uint32_t SM_MISC = SM_BAR + 512;
-constexpr uint32_t SM_TOTAL = SM_MISC + 64;
+constexpr uint32_t SM_PSF = SM_MISC + 128;                   // scale atom of the 4-bit P (512 B)
+constexpr uint32_t SM_Q4 = (SM_PSF + 512 + 1023) & ~1023u;   // NVFP4 Q of the pair [128][64 B], SW64
+constexpr uint32_t SM_TOTAL = SM_Q4 + 8192;
+// 4-bit unit: K slot = K4 [64][64 B] SW64 at +0, its scale atoms (2 x 512 B) at
+// +8192; V slot = V4^T [128][32 B] SW32 at +0, its scale atom at +8192
+constexpr uint32_t SL_SF = 8192;
 constexpr uint32_t kSmemBytes = SM_TOTAL + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns: O 0-127, S 2 x 128 at 128 (a 16-bit unit fills 128, an INT8
-// unit 64), X 128 at 384
+// TMEM columns: O 0-127, S 2 x 128 at 128 (a 16-bit unit fills 128, an INT8 or
+// 4-bit unit 64), X 128 at 384.  4-bit units keep their scale factors in the
+// upper half of their S buffer: K scales at +64, V scales at +72, P scales at
+// +76; Q's scales (constant for the CTA) at 216.  Scale columns are 4-aligned.
 constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384;
+constexpr uint32_t TM_SFQ = 216, TMO_SFK = 64, TMO_SFV = 72, TMO_SFP = 76;
 
 // mbarrier slots (8 bytes each)
 enum {
-  B_Q16 = 0, B_Q8, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
+  B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
   B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages,
   B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_X_FULL = B_P_FREE + 1,
   B_X_FREE = B_X_FULL + 1, B_DONE = B_X_FREE + 1,
@@ -96,6 +110,10 @@ struct TcArgs {
   const float* q_s8;
   const float* k_s8;
   const float* v_s8;
+  const float* v_g4;
+  const uint8_t* q_sf4;
+  const uint8_t* k_sf4;
+  const uint8_t* v_sf4;
   int* status;
   int npairs;
 };
@@ -166,7 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const __grid_constant__ CUtensorMap tmQ8, const __grid_constant__ CUtensorMap tmK8,
-               const __grid_constant__ CUtensorMap tmV8, Geom g, TcArgs A) {
+               const __grid_constant__ CUtensorMap tmV8, const __grid_constant__ CUtensorMap tmQ4,
+               const __grid_constant__ CUtensorMap tmK4, const __grid_constant__ CUtensorMap tmV4, Geom g,
+               TcArgs A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s0 = (uint32_t)__cvta_generic_to_shared(smem);
@@ -175,8 +195,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int qa = 2 * pair, qb = (2 * pair + 1 < g.nb) ? 2 * pair + 1 : -1;
   const size_t prow = (size_t)bh * A.npairs + pair;
   const int4 pc = *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
-  const int n16 = pc.x, n8 = pc.y;
-  const int n = n16 + n8;
+  const int n16 = pc.x, n8 = pc.y, n4 = pc.z;
   const uint32_t* items = A.plist + prow * (size_t)(2 * g.nb);
   auto bar = [&](int i) { return s0 + SM_BAR + 8u * (uint32_t)i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM_MISC);
@@ -185,15 +204,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // units: 16-bit items are taken two at a time (one N = 128 score MMA per
   // unit), INT8 items one at a time
   const int nu16 = (n16 + 1) / 2;
-  const int nu = nu16 + n8;
+  const int nu8 = nu16 + n8;  // INT8 units end here, 4-bit units follow
+  const int nu = nu8 + n4;
   auto unit_items = [&](int u, int& i0, int& cnt) {
     if (u < nu16) { i0 = 2 * u; cnt = min(2, n16 - 2 * u); }
-    else { i0 = n16 + (u - nu16); cnt = 1; }
+    else { i0 = n16 + (u - nu16); cnt = 1; }  // INT8 and 4-bit items follow in list order
   };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q16), 1);
     mbar_init(bar(B_Q8), 1);
+    mbar_init(bar(B_Q4), 1);
+    mbar_init(bar(B_SFQ), 4);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(B_K_FULL + s), 1); mbar_init(bar(B_K_EMPTY + s), 1);
       mbar_init(bar(B_V_FULL + s), 1); mbar_init(bar(B_V_EMPTY + s), 1);
@@ -213,7 +235,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(s0 + SM_MISC, 512);
-  if (threadIdx.x < kD) reinterpret_cast<float*>(smem + SM_VS)[threadIdx.x] = A.v_s8[(size_t)bh * kD + threadIdx.x];
+  if (threadIdx.x < kD) {
+    reinterpret_cast<float*>(smem + SM_VS)[threadIdx.x] = A.v_s8[(size_t)bh * kD + threadIdx.x];
+    reinterpret_cast<float*>(smem + SM_VS + 512)[threadIdx.x] = A.v_g4[(size_t)bh * kD + threadIdx.x];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -247,6 +272,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_2d(s0 + SM_Q8, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qa) * 64);
         if (qb >= 0) tma_load_2d(s0 + SM_Q8 + 8192, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qb) * 64);
       }
+      if (n4 > 0) {
+        mbar_expect_tx(bar(B_Q4), qb >= 0 ? 8192u : 4096u);
+        tma_load_2d(s0 + SM_Q4, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qa) * 64);
+        if (qb >= 0) tma_load_2d(s0 + SM_Q4 + 4096, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qb) * 64);
+      }
       // K of a unit is needed first (scores) and released first; V waits for
       // the P·V two units back.  Issue whichever ring has room, K first.
       int kn = 0, vn = 0;
@@ -265,9 +295,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_4d(dst + t * 8192, &tmK, fb, 0, cx, cy, cf);
               tma_load_4d(dst + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
             }
-          } else {
+          } else if (kn < nu8) {
             mbar_expect_tx(fb, 8192u);
             tma_load_2d(dst, &tmK8, fb, 0, (bh * g.nb + item_kb(items[i0])) * 64);
+          } else {
+            const size_t kl = (size_t)bh * g.nb + item_kb(items[i0]);
+            mbar_expect_tx(fb, 4096u + 1024u);
+            tma_load_2d(dst, &tmK4, fb, 0, (int)(kl * 64));
+            bulk_load(dst + SL_SF, A.k_sf4 + kl * 2 * kSfAtomBytes, 2 * kSfAtomBytes, fb);
           }
           ++kn;
           progressed = true;
@@ -284,9 +319,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_4d(dst + t * 16384, &tmV, fb, 0, cx, cy, cf);
               tma_load_4d(dst + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
             }
-          } else {
+          } else if (vn < nu8) {
             mbar_expect_tx(fb, 8192u);
             tma_load_2d(dst, &tmV8, fb, 0, (bh * g.nb + item_kb(items[i0])) * kD);
+          } else {
+            const size_t kl = (size_t)bh * g.nb + item_kb(items[i0]);
+            mbar_expect_tx(fb, 4096u + kSfAtomBytes);
+            tma_load_2d(dst, &tmV4, fb, 0, (int)(kl * kD));
+            bulk_load(dst + SL_SF, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
           }
           ++vn;
           progressed = true;
@@ -307,6 +347,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t idpv = idesc(kDF32, kFmtBF16, kFmtBF16, false, true, 128, 128);
       const uint32_t id8 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
       const uint32_t idx8 = idesc(kDS32, kFmtU8, kFmtS8, false, false, 128, 128);
+      const uint32_t id4s = idesc_f4(128, 64), id4pv = idesc_f4(128, 128);
+      bool f4_ready = false;  // Q4 loaded and its scales in TMEM
       bool ok = true;
       if (n16 > 0) ok = ok && mbar_wait(bar(B_Q16), 0);
       if (n8 > 0) ok = ok && mbar_wait(bar(B_Q8), 0);
@@ -316,7 +358,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         bool progressed = false;
         if (sn < nu) {
           const int s = sn % kStages, b = sn & 1;
-          if (mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1) &&
+          if (sn >= nu8 && !f4_ready) {
+            // first 4-bit unit: Q4 must be in shared memory and its scales in TMEM
+            f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
+          }
+          if ((sn < nu8 || f4_ready) && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1) &&
               (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1))) {
             tc_fence_after();
             const uint32_t st = s0 + SM_K + s * 32768;
@@ -331,11 +377,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 mma_f16(sd, smem_desc(s0 + SM_Q16 + h * 16384 + kk * 32, 16, 1024, SW_128),
                         smem_desc(st + h * 16384 + kk * 32, 16, 1024, SW_128), id, k > 0 ? 1u : 0u);
               }
-            } else {
+            } else if (sn < nu8) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
                        smem_desc(st + kk * 32, 16, 1024, SW_128), id8, kk > 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                tc_cp_atom(sd + TMO_SFK + 4 * c, st + SL_SF + c * kSfAtomBytes);
+                mma_f4(sd, smem_desc(s0 + SM_Q4 + 32 * c, 16, 512, SW_64), smem_desc(st + 32 * c, 16, 512, SW_64),
+                       id4s, c > 0 ? 1u : 0u, tbase + TM_SFQ + 4 * c, sd + TMO_SFK + 4 * c);
+              }
             }
             mma_commit(bar(B_S_FULL + b));
             mma_commit(bar(B_K_EMPTY + s));
@@ -345,7 +398,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (pn < sn) {
           const int s = pn % kStages;
-          const bool int8 = pn >= nu16;
+          const bool int8 = pn >= nu16;  // INT8 or 4-bit: both produce a block result X
           if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL), pn & 1) &&
               (!int8 || xu < 1 || mbar_test(bar(B_X_FREE), (xu - 1) & 1))) {
             tc_fence_after();
@@ -360,11 +413,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                   mma_f16(tbase + TM_O, smem_desc(pbuf + t * 16384 + kk * 32, 16, 1024, SW_128),
                           smem_desc(st + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
               }
-            } else {
+            } else if (pn < nu8) {
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk)
                 mma_i8(tbase + TM_X, smem_desc(pbuf + kk * 32, 16, 512, SW_64),
                        smem_desc(st + kk * 32, 16, 512, SW_64), idx8, kk > 0 ? 1u : 0u);
+              mma_commit(bar(B_X_FULL));
+              ++xu;
+            } else {
+              const uint32_t sfb = tbase + TM_S + (pn & 1) * 128;
+              tc_cp_atom(sfb + TMO_SFV, st + SL_SF);
+              tc_cp_atom(sfb + TMO_SFP, s0 + SM_PSF);
+              mma_f4(tbase + TM_X, smem_desc(pbuf, 16, 256, SW_32), smem_desc(st, 16, 256, SW_32), id4pv, 0u,
+                     sfb + TMO_SFP, sfb + TMO_SFV);
               mma_commit(bar(B_X_FULL));
               ++xu;
             }
@@ -552,7 +613,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return true;
     };
 
-    for (int u = nu16; ok && u < nu; ++u) {
+    for (int u = nu16; ok && u < nu8; ++u) {
       if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
       const int b = u & 1;
       int i0, cnt;
@@ -650,10 +711,186 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         pend_lb = lb;
     }
     if (ok && have_pend) ok = merge_x();
+    const float* vsc = reinterpret_cast<const float*>(smem + SM_VS);  // scale of the register accumulator
+    if (ok && n4 > 0) {
+      // ---- phase boundary 8 -> 4: fold the INT8 accumulator into O with its
+      // channel scale, so the registers can carry the 4-bit phase
+      if (n8 > 0) {
+        const float mm = fmaxf(m16, m8);
+        const float a16 = m16 == -INFINITY ? 0.f : fast_exp2(m16 - mm);
+        const float a8 = m8 == -INFINITY ? 0.f : fast_exp2(m8 - mm);
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t orr[32];
+          tmem_ld32(tbase + lane_off + TM_O + half * 64 + c, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            orr[i] = __float_as_uint(a16 * __uint_as_float(orr[i]) + a8 * vs[half * 64 + c + i] * o8[c + i]);
+          tmem_st32(tbase + lane_off + TM_O + half * 64 + c, orr);
+        }
+        tmem_wait_st();
+        l16 = l16 * a16 + l8 * a8;
+        m16 = mm;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) o8[i] = 0.f;
+        m8 = -INFINITY;
+        l8 = 0.f;
+      }
+      // Q's scale factors into TMEM (each lane quarter holds all 128 rows)
+      if (half == 0) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w[4];
+          const uint8_t* sa = A.q_sf4 + ((size_t)bh * g.nb + qa) * 2 * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+          w[0] = *reinterpret_cast<const uint32_t*>(sa);
+          w[1] = *reinterpret_cast<const uint32_t*>(sa + 4);
+          if (qb >= 0) {
+            const uint8_t* sb = A.q_sf4 + ((size_t)bh * g.nb + qb) * 2 * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+            w[2] = *reinterpret_cast<const uint32_t*>(sb);
+            w[3] = *reinterpret_cast<const uint32_t*>(sb + 4);
+          } else {
+            w[2] = w[3] = 0u;
+          }
+          tmem_st4(tbase + lane_off + TM_SFQ + 4 * c, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SFQ));
+      }
+      vsc = reinterpret_cast<const float*>(smem + SM_VS + 512);  // g
+      // fold a 4-bit block result X (fp32) into the register accumulator
+      auto merge_x4 = [&]() -> bool {
+        if (!__all_sync(FULL, mbar_wait(bar(B_X_FULL), xu & 1))) return false;
+        tc_fence_after();
+        if (pend_member) {
+          uint32_t xr[64];
+          tmem_ld32(tbase + lane_off + TM_X + half * 64, xr);
+          tmem_ld32(tbase + lane_off + TM_X + half * 64 + 32, xr + 32);
+          tmem_wait_ld();
+          if (pend_mb > m8 + kRescaleThreshold || m8 == -INFINITY) {
+            const float nm = ceilf(pend_mb);
+            const float a = (m8 == -INFINITY) ? 0.f : ldexpf(1.0f, (int)(m8 - nm));
+#pragma unroll
+            for (int i = 0; i < 64; ++i) o8[i] *= a;
+            l8 *= a;
+            m8 = nm;
+          }
+          const float f = fast_exp2(pend_mb - m8);
+          l8 += pend_lb * f;
+          const uint64_t fx2 = f2pack(f, f);
+#pragma unroll
+          for (int i = 0; i < 64; i += 2)
+            f2unpack(f2fma(fx2, f2pack(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), f2pack(o8[i], o8[i + 1])),
+                     o8[i], o8[i + 1]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_X_FREE));
+        ++xu;
+        have_pend = false;
+        return true;
+      };
+      for (int u = nu8; ok && u < nu; ++u) {
+        if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+        const int b = u & 1;
+        int i0, cnt;
+        unit_items(u, i0, cnt);
+        float* xch = red + (u & 1) * 256;
+        const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
+        // ---- 4-bit unit: one key block; this warp owns keys 32*half..+31
+        const uint32_t e = items[i0];
+        const int kb = item_kb(e);
+        const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
+        if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(sbase + half * 32, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
+        const unsigned long long vm = item_full(e) ? ~0ull : (key_mask(g, kb) >> (32 * half));
+        const bool full = (uint32_t)vm == 0xffffffffu;
+        float mx = -INFINITY;
+        if (member) {
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
+          }
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
+          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        }
+        xch[half * 128 + row] = mx;
+        if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+        mx = fmaxf(mx, xch[(1 - half) * 128 + row]);
+        float mb = -INFINITY, lb = 0.f;
+        uint32_t pw[4] = {0u, 0u, 0u, 0u};
+        uint32_t sfw = 0u;  // this half-row's two e4m3 P scales
+        if (member) {
+          mb = mx * sl2;
+          float pv[32];
+          const uint64_t sl2x2 = f2pack(sl2, sl2), negm = f2pack(-mb, -mb);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            f2unpack(f2fma(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm), x0, x1);
+            pv[2 * i] = fast_exp2(x0);
+            pv[2 * i + 1] = fast_exp2(x1);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) lb += pv[i];
+          // NVFP4 over 16 consecutive keys: e4m3 scale from the microblock max / 6
+#pragma unroll
+          for (int mbk = 0; mbk < 2; ++mbk) {
+            float pm = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pm = fmaxf(pm, pv[16 * mbk + i]);
+            const uint32_t sf = cvt_e4m3x2(0.0f, __fdiv_rn(pm, 6.0f)) & 0xffu;
+            sfw |= sf << (8 * mbk);
+            const float dec = e4m3_to_f32(sf);
+            if (dec != 0.f) {
+              const float r = __fdiv_rn(1.0f, dec);
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                uint32_t w = 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  const int k = 16 * mbk + 8 * q + 2 * t;
+                  w |= cvt_e2m1x2(__fmul_rn(pv[k + 1], r), __fmul_rn(pv[k], r)) << (8 * t);
+                }
+                pw[2 * mbk + q] = w;
+              }
+            }
+          }
+        }
+        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        *reinterpret_cast<uint4*>(smem + SM_P + row * 32 + ((half ^ ((row >> 2) & 1)) * 16)) =
+            make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        *reinterpret_cast<uint16_t*>(smem + SM_PSF + (row & 31) * 16 + (row >> 5) * 4 + 2 * half) = (uint16_t)sfw;
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_P_FULL));
+        if (have_pend && !merge_x4()) { ok = false; break; }
+        have_pend = true;
+        pend_member = member;
+        pend_mb = mb;
+        pend_lb = lb;
+      }
+      if (ok && have_pend) ok = merge_x4();
+    }
     if (ok && !__all_sync(FULL, mbar_wait(bar(B_DONE), 0))) ok = false;
     tc_fence_after();
     if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
-    // ---- phase boundary and epilogue: O = (2^(m16-m) O16 + 2^(m8-m) sv ⊙ o8) / l
+    // ---- epilogue: O = (2^(m16-m) O + 2^(m8-m) vsc ⊙ o8) / l, vsc the channel
+    // scale of whichever low-bit phase ran last (INT8 sv or NVFP4 g)
     {
       // both halves of a row carry partial sums; exchange them
       float* lx = red + 512;  // [2 halves][2 values][128 rows], past the item buffers
@@ -677,8 +914,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int ch = half * 64 + c + 2 * i;
-          const float v0 = (a16 * __uint_as_float(orr[2 * i]) + a8 * vs[ch] * o8[c + 2 * i]) * il;
-          const float v1 = (a16 * __uint_as_float(orr[2 * i + 1]) + a8 * vs[ch + 1] * o8[c + 2 * i + 1]) * il;
+          const float v0 = (a16 * __uint_as_float(orr[2 * i]) + a8 * vsc[ch] * o8[c + 2 * i]) * il;
+          const float v1 = (a16 * __uint_as_float(orr[2 * i + 1]) + a8 * vsc[ch + 1] * o8[c + 2 * i + 1]) * il;
           __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
           w[i] = *reinterpret_cast<uint32_t*>(&hb);
         }
@@ -817,7 +1054,7 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t rowbytes
 }  // namespace
 
 bool attention_tc_supported(const Geom& g) {
-  return g.d == kD && g.n4 == 0 && encode_fn() != nullptr;
+  return g.d == kD && encode_fn() != nullptr;
 }
 
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st) {
@@ -829,12 +1066,15 @@ cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStre
 
 cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, const void* k, const void* v,
                                 void* ws, void* out, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, to, tq8, tk8, tv8;
+  CUtensorMap tq, tk, tv, to, tq8, tk8, tv8, tq4, tk4, tv4;
   const uint64_t rows64 = (uint64_t)g.BH * g.nb * 64, rows128 = (uint64_t)g.BH * g.nb * kD;
   if (!map_regions(&tq, q, g) || !map_regions(&tk, k, g) || !map_regions(&tv, v, g) || !map_regions(&to, out, g) ||
       !map_rows(&tq8, at<int8_t>(ws, L, R_Q_I8), rows64, kD, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !map_rows(&tk8, at<int8_t>(ws, L, R_K_I8), rows64, kD, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map_rows(&tv8, at<int8_t>(ws, L, R_V_I8), rows128, 64, kD, CU_TENSOR_MAP_SWIZZLE_64B))
+      !map_rows(&tv8, at<int8_t>(ws, L, R_V_I8), rows128, 64, kD, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map_rows(&tq4, at<uint8_t>(ws, L, R_Q_F4), rows64, kD / 2, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map_rows(&tk4, at<uint8_t>(ws, L, R_K_F4), rows64, kD / 2, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map_rows(&tv4, at<uint8_t>(ws, L, R_V_F4), rows128, 32, kD, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
   cudaError_t e = launch_pair_lists(g, L, ws, st);
   if (e != cudaSuccess) return e;
@@ -845,11 +1085,16 @@ cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, c
   A.q_s8 = at<float>(ws, L, R_Q_S8);
   A.k_s8 = at<float>(ws, L, R_K_S8);
   A.v_s8 = at<float>(ws, L, R_V_S8);
+  A.v_g4 = at<float>(ws, L, R_V_G4);
+  A.q_sf4 = at<uint8_t>(ws, L, R_Q_SF4);
+  A.k_sf4 = at<uint8_t>(ws, L, R_K_SF4);
+  A.v_sf4 = at<uint8_t>(ws, L, R_V_SF4);
   A.status = status;
   A.npairs = (g.nb + 1) / 2;
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq8, tk8, tv8, g, A);
+  attn_tc_kernel<<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq8, tk8, tv8, tq4, tk4, tv4,
+                                                                      g, A);
   return cudaGetLastError();
 }
 

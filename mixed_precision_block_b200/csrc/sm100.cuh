@@ -171,6 +171,30 @@ __device__ __forceinline__ void mma_i8(uint32_t dtmem, uint64_t adesc, uint64_t 
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(id), "r"(acc));
 }
+// kind::mxf4nvf4 (e2m1 x e2m1, ue4m3 scale per 16 elements along K, K = 64 per
+// instruction, fp32 D).  Instruction descriptor for block-scaled kinds:
+//   [7,10) A format (e2m1 = 1)  [10,13) B format  [17,23) N >> 3  [23] scale
+//   format (ue4m3 = 0)  [24,29) M >> 4; both scale-factor ids 0.
+__host__ __device__ constexpr uint32_t idesc_f4(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// sfa / sfb: TMEM addresses (4-column aligned) of the scale factors, laid out
+// as the copy atom: per 64-element chunk, lane i of every lane quarter holds
+// the scales of rows i, i+32, i+64, i+96 in four consecutive columns.
+__device__ __forceinline__ void mma_f4(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t id, uint32_t acc,
+                                       uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(id), "r"(acc), "r"(sfa), "r"(sfb));
+}
+// Copy one 32-line x 16-byte scale atom from shared memory into TMEM,
+// replicated into the four lane quarters (ordered with later MMAs).
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint32_t saddr) {
+  const uint64_t d = smem_desc(saddr, 16, 128, SW_NONE);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d));
+}
+
 // Arrives once on `bar` when every MMA issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
