@@ -51,13 +51,14 @@ def phase_flops(wl, info):
     return {16: per_pair * info.n16 * bh, 8: per_pair * info.n8 * bh, 4: per_pair * info.n4 * bh}
 
 
-def launches_per_call(info):
+def launches_per_call(info, d):
     """Kernels this library launches per call (its own kernels only)."""
     v = 2 if (info.n8 or info.n4) else 0  # v_amax + pack_v
     prep = 1 + v
     draft = 2  # logits + mix (mix carries the first ranking histogram)
     rank = 1 + 8 + 7 + 1  # init, 8 selects, 7 histogram passes, assign
-    return prep + draft + rank + 1
+    attn = 2 if d == 128 else 1  # pair lists + tensor-core kernel, or the warp-MMA kernel
+    return prep + draft + rank + attn
 
 
 class ClockSampler:
@@ -199,10 +200,15 @@ def config_of(wl, args):
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
 
 
-def traffic_record(kernel_src):
+def roofline_kernel(wl):
+    """(kernel name, source file) of the attention kernel the call runs."""
+    return ("attn_tc_kernel", "attn_tc.cu") if wl.d == 128 else ("attn_mp_kernel", "attn.cu")
+
+
+def traffic_record(kernel, kernel_src, workload):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     summary, or None if the kernel source changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", "attn_mp_video_traffic.json")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -326,7 +332,8 @@ def run_ours(args, wl):
     attn_ms = stage[2]
     achieved = f_tot / (attn_ms * 1e-3) / 1e12
     peak_blend = f_tot / t_roof_s / 1e12
-    traffic = traffic_record(os.path.join(ROOT, "mixed_precision_block_b200", "csrc", "attn.cu"))
+    kname, ksrc = roofline_kernel(wl)
+    traffic = traffic_record(kname, os.path.join(ROOT, "mixed_precision_block_b200", "csrc", ksrc), wl.name)
     clocks = clk.summary()
 
     if rank == 0:
@@ -342,14 +349,13 @@ def run_ours(args, wl):
             "stages_ms": {"prepare": stage[0], "draft_rank": stage[1], "attention": stage[2]},
             "dense_bf16": {"ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
                            "speedup_of_sparse_call": dense_ms / ms},
-            "roofline": {"bound": "tensor", "kernel": ("attn_tc_kernel" if wl.d == 128 and info.n4 == 0
-                                                        else "attn_mp_kernel"), "achieved": achieved,
+            "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved,
                          "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
                          "traffic": traffic,
                          "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
                                       f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
                                       f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"},
-            "e2e": e2e, "gpu_launches": launches_per_call(info) * args.steps, "clocks": clocks,
+            "e2e": e2e, "gpu_launches": launches_per_call(info, wl.d) * args.steps, "clocks": clocks,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
