@@ -281,16 +281,19 @@ def run_ours(args, wl):
     value = world * flops / (ms * 1e-3) / 1e12
 
     # own dense bf16 kernel on the same inputs
-    dense_out = torch.empty_like(q)
-    with torch.cuda.stream(st):
-        da2.da2_dense_attention(q, k, v, dense_out, st)
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(st)
-        for _ in range(args.dense_steps):
+    dense_ms = None
+    if args.dense_steps > 0:
+        dense_out = torch.empty_like(q)
+        with torch.cuda.stream(st):
             da2.da2_dense_attention(q, k, v, dense_out, st)
-        d1.record(st)
-    torch.cuda.synchronize(dev)
-    dense_ms = d0.elapsed_time(d1) / args.dense_steps
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(st)
+            for _ in range(args.dense_steps):
+                da2.da2_dense_attention(q, k, v, dense_out, st)
+            d1.record(st)
+        torch.cuda.synchronize(dev)
+        dense_ms = d0.elapsed_time(d1) / args.dense_steps
+        del dense_out
 
     # end to end through host buffers: pinned H2D of Q/K/V, the call, D2H of O
     e2e = None
@@ -347,8 +350,9 @@ def run_ours(args, wl):
             "vs_baseline": None, "dtype": "bf16+int8+nvfp4 (fp32 accumulate)", "data": "synthetic",
             "config": config_of(wl, args),
             "stages_ms": {"prepare": stage[0], "draft_rank": stage[1], "attention": stage[2]},
-            "dense_bf16": {"ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
-                           "speedup_of_sparse_call": dense_ms / ms},
+            "dense_bf16": None if dense_ms is None else {
+                "ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
+                "speedup_of_sparse_call": dense_ms / ms},
             "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved,
                          "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
                          "traffic": traffic,
@@ -372,6 +376,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="video")
     ap.add_argument("--lam", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None, help="run only this many heads (profiling captures)")
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-frames", type=int, default=2, help="frames per CPU oracle sample (reference arm)")
@@ -384,6 +389,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.lam is not None:
         wl = wl.with_(lam=args.lam)
+    if args.heads is not None:
+        wl = wl.with_(H=args.heads)
     if args.impl == "reference":
         run_reference(args, wl)
     else:
