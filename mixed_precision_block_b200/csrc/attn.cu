@@ -13,14 +13,19 @@
 //   phase 16  bf16 Q/K/V tiles gathered from the [B,H,N,d] inputs (8 rows of 8
 //             contiguous tokens per region), cp.async double-buffered,
 //             m16n8k16 bf16 MMAs, online softmax, P in bf16.
+//   The low-bit phases walk the key blocks in units of two, as the
+//   tensor-core kernel does for the query-block pair (2p, 2p+1): per unit the
+//   row maximum over the member blocks comes first (scores only), raising the
+//   phase's power-of-two P reference 2^r to ceil(max) where the max exceeds
+//   it; then each member block is scored again and its P quantised against 2^r.
 //   phase 8   INT8 Q/K codes with block scales (m16n8k32 s8·s8 → s32);
-//             P = round(255·exp(s − m_blk)) as u8 through shared memory;
+//             P = round(255·2^(x − r)) as u8 through shared memory;
 //             P·V on u8·s8 codes; int32 block result scaled by
-//             exp(m_blk − m)/255 and the per-channel V scale when merged.
+//             2^(r − m)/255 and the per-channel V scale when merged.
 //   phase 4   NVFP4 codes dequantised exactly to f16 in shared memory
-//             (e2m1 × e4m3 fits f16), m16n8k16 f16 MMAs, P re-quantised to
-//             NVFP4 per 16 keys in registers, block result scaled by
-//             exp(m_blk − m) and the per-channel V scale g when merged.
+//             (e2m1 × e4m3 fits f16), m16n8k16 f16 MMAs, 2688·P
+//             re-quantised to NVFP4 per 16 keys in registers, block result
+//             scaled by 2^(r − m)/2688 and the per-channel V scale g when merged.
 // attn_dense: the phase-16 path over all tokens in natural order.
 #include "da2_internal.cuh"
 #include "mma_sm80.cuh"
@@ -56,6 +61,8 @@ struct AttnArgs {
   const float* v_g4;
   const uint16_t* lists;
   const int* counts;
+  const uint32_t* plist;  // merged key lists of the query-block pairs
+  const int* pcnt;
 };
 
 // Real-token mask of a region block's 64 slots.
@@ -246,13 +253,15 @@ __device__ __forceinline__ void merge_block(float (*O)[4], float* m, float* l, f
   }
 }
 
-// Block-local softmax numerators: p = exp2(s - m_blk); returns the row sums.
-__device__ __forceinline__ void block_probs(float (*S)[4], float mb0, float mb1, float& lb0, float& lb1) {
+// Softmax numerators against the phase reference: p = exp2(s - r) (0 for a row
+// with no reference yet); returns the row sums.
+__device__ __forceinline__ void block_probs(float (*S)[4], float r0, float r1, float& lb0, float& lb1) {
   float s0 = 0.f, s1 = 0.f;
+  const bool ok0 = r0 != -INFINITY, ok1 = r1 != -INFINITY;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    S[j][0] = fast_exp2(S[j][0] - mb0); S[j][1] = fast_exp2(S[j][1] - mb0);
-    S[j][2] = fast_exp2(S[j][2] - mb1); S[j][3] = fast_exp2(S[j][3] - mb1);
+    S[j][0] = ok0 ? fast_exp2(S[j][0] - r0) : 0.f; S[j][1] = ok0 ? fast_exp2(S[j][1] - r0) : 0.f;
+    S[j][2] = ok1 ? fast_exp2(S[j][2] - r1) : 0.f; S[j][3] = ok1 ? fast_exp2(S[j][3] - r1) : 0.f;
     s0 += S[j][0] + S[j][1];
     s1 += S[j][2] + S[j][3];
   }
@@ -260,13 +269,10 @@ __device__ __forceinline__ void block_probs(float (*S)[4], float mb0, float mb1,
   lb1 = quad_sum(s1);
 }
 
-// One INT8 key block.
+// INT8 scores of one key block (exact integers, as floats).
 template <int D>
-__device__ __forceinline__ void block8(uint32_t sQ, uint32_t sK, uint32_t sV, uint8_t* sPw,
-                                       unsigned long long vmask, float sc, int warp, int lane,
-                                       float (*O)[4], float* m, float* l, const float* vscale) {
+__device__ __forceinline__ void qk_int8(uint32_t sQ, uint32_t sK, int warp, int lane, float (*S)[4]) {
   constexpr int QCPR = D / 16;  // INT8 Q/K rows: D bytes
-  const int gq = lane >> 2, tq = lane & 3;
   int Si[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j) Si[j][0] = Si[j][1] = Si[j][2] = Si[j][3] = 0;
@@ -284,14 +290,24 @@ __device__ __forceinline__ void block8(uint32_t sQ, uint32_t sK, uint32_t sV, ui
       mma_s8s8(Si[2 * np + 1], a, b2, b3);
     }
   }
-  float S[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
 #pragma unroll
     for (int e = 0; e < 4; ++e) S[j][e] = (float)Si[j][e];
-  float mb0, mb1, lb0, lb1;
-  scale_mask(S, sc, vmask, tq, mb0, mb1);
-  block_probs(S, mb0, mb1, lb0, lb1);
+}
+
+// One INT8 key block, P quantised against the phase reference r (2 rows).
+template <int D>
+__device__ __forceinline__ void block8(uint32_t sQ, uint32_t sK, uint32_t sV, uint8_t* sPw,
+                                       unsigned long long vmask, float sc, int warp, int lane,
+                                       float (*O)[4], float* m, float* l, const float* vscale,
+                                       const float* r) {
+  const int gq = lane >> 2, tq = lane & 3;
+  float S[8][4];
+  qk_int8<D>(sQ, sK, warp, lane, S);
+  float mx0, mx1, lb0, lb1;
+  scale_mask(S, sc, vmask, tq, mx0, mx1);
+  block_probs(S, r[0], r[1], lb0, lb1);
   // u8 P codes, round(255 p), through this warp's [16][64] shared tile
   const uint32_t sP = smem_u32(sPw);
 #pragma unroll
@@ -320,13 +336,15 @@ __device__ __forceinline__ void block8(uint32_t sQ, uint32_t sK, uint32_t sV, ui
     }
   }
   __syncwarp();
-  merge_block<D, int>(O, m, l, mb0, mb1, lb0, lb1, X, 1.0f / 255.0f, vscale, tq);
+  merge_block<D, int>(O, m, l, r[0], r[1], lb0, lb1, X, 1.0f / 255.0f, vscale, tq);
 }
 
-// NVFP4 re-quantisation of 4 probabilities of one row's 16-key microblock
-// (this lane's 4, the other 12 in the lane quad) → two f16x2 A-fragment words.
+// NVFP4 re-quantisation of 2688 p for 4 probabilities of one row's 16-key
+// microblock (this lane's 4, the other 12 in the lane quad) → two f16x2
+// A-fragment words holding the dequantised values (2688 p, quantised).
 __device__ __forceinline__ void quant_p4(float p0, float p1, float p2, float p3, uint32_t& w01,
                                          uint32_t& w23) {
+  p0 *= 2688.0f; p1 *= 2688.0f; p2 *= 2688.0f; p3 *= 2688.0f;
   float mx = fmaxf(fmaxf(p0, p1), fmaxf(p2, p3));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -343,17 +361,18 @@ __device__ __forceinline__ void quant_p4(float p0, float p1, float p2, float p3,
   w23 = *reinterpret_cast<uint32_t*>(&hb);
 }
 
-// One NVFP4 key block (K and V^T already dequantised to f16 in shared memory).
+// One NVFP4 key block (K and V^T already dequantised to f16 in shared memory),
+// P quantised against the phase reference r (2 rows).
 template <int D>
 __device__ __forceinline__ void block4(uint32_t sQ, uint32_t sK, uint32_t sVt, unsigned long long vmask,
                                        float sl2, int warp, int lane, float (*O)[4], float* m, float* l,
-                                       const float* vscale) {
+                                       const float* vscale, const float* r) {
   const int tq = lane & 3;
   float S[8][4];
   qk_16bit<D, true>(sQ, sK, warp, lane, S);
-  float mb0, mb1, lb0, lb1;
-  scale_mask(S, sl2, vmask, tq, mb0, mb1);
-  block_probs(S, mb0, mb1, lb0, lb1);
+  float mx0, mx1, lb0, lb1;
+  scale_mask(S, sl2, vmask, tq, mx0, mx1);
+  block_probs(S, r[0], r[1], lb0, lb1);
   float X[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) X[n][0] = X[n][1] = X[n][2] = X[n][3] = 0.f;
@@ -372,7 +391,7 @@ __device__ __forceinline__ void block4(uint32_t sQ, uint32_t sK, uint32_t sVt, u
       mma_f16(X[2 * np + 1], a, b2, b3);
     }
   }
-  merge_block<D, float>(O, m, l, mb0, mb1, lb0, lb1, X, 1.0f, vscale, tq);
+  merge_block<D, float>(O, m, l, r[0], r[1], lb0, lb1, X, 1.0f / 2688.0f, vscale, tq);
 }
 
 // Normalise, round to bf16, and write this warp's 16 rows to their tokens.
@@ -438,56 +457,99 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_mp_kernel(Geom g, AttnAr
       __syncthreads();
     }
   }
+  // units of the low-bit phases: the pair's merged key lists, two entries at a
+  // time; this query block takes the entries it is a member of
+  const size_t prow = (size_t)bh * ((g.nb + 1) / 2) + (qb >> 1);
+  const int4 pc = *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
+  const uint32_t* items = A.plist + prow * (size_t)(2 * g.nb);
+  const int mbit = (qb & 1) ? 17 : 16;
+  auto unit_members = [&](const uint32_t* it, int n, int i, int* kbs) {
+    int nm = 0;
+    for (int t = 0; t < 2 && i + t < n; ++t) {
+      const uint32_t e = it[i + t];
+      if ((e >> mbit) & 1u) kbs[nm++] = (int)(e & 0xffffu);
+    }
+    return nm;
+  };
+  // raise the phase reference to ceil(unit max) where the max exceeds it
+  auto raise_ref = [&](float* r, float ux0, float ux1) {
+    if (ux0 != -INFINITY && (r[0] == -INFINITY || ux0 > r[0])) r[0] = ceilf(ux0);
+    if (ux1 != -INFINITY && (r[1] == -INFINITY || ux1 > r[1])) r[1] = ceilf(ux1);
+  };
+  const int tq = lane & 3;
   // ---------------- phase 8
   if (cnt.y > 0) {
-    const uint16_t* l8 = list + cnt.x;
     load_bytes_swz<D>(s0 + SL::Q, reinterpret_cast<const uint8_t*>(A.q_i8) + row_lin * 64 * D, 64);
     for (int c = threadIdx.x; c < D; c += kAttnThreads) vs[c] = A.v_s8[(size_t)bh * D + c];
     const float sq = A.q_s8[row_lin];
-    auto issue = [&](int j) {
-      const size_t kl = (size_t)bh * g.nb + l8[j];
-      load_bytes_swz<D>(s0 + SL::K + (j & 1) * SL::TILE16,
-                        reinterpret_cast<const uint8_t*>(A.k_i8) + kl * 64 * D, 64);
-      load_bytes_swz<64>(s0 + SL::V + (j & 1) * SL::TILE16,
-                         reinterpret_cast<const uint8_t*>(A.v_i8) + kl * 64 * D, D);
+    float r[2] = {-INFINITY, -INFINITY};
+    const uint32_t* it8 = items + pc.x;
+    for (int i = 0; i < pc.y; i += 2) {
+      int kbs[2];
+      const int nm = unit_members(it8, pc.y, i, kbs);
+      if (nm == 0) continue;
+      for (int t = 0; t < nm; ++t) {
+        const size_t kl = (size_t)bh * g.nb + kbs[t];
+        load_bytes_swz<D>(s0 + SL::K + t * SL::TILE16, reinterpret_cast<const uint8_t*>(A.k_i8) + kl * 64 * D, 64);
+        load_bytes_swz<64>(s0 + SL::V + t * SL::TILE16, reinterpret_cast<const uint8_t*>(A.v_i8) + kl * 64 * D, D);
+      }
       cp_async_commit();
-    };
-    issue(0);
-    for (int j = 0; j < cnt.y; ++j) {
-      if (j + 1 < cnt.y) { issue(j + 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
+      cp_async_wait<0>();
       __syncthreads();
-      const int kb = l8[j];
-      const float sc = sq * A.k_s8[(size_t)bh * g.nb + kb] * sl2;
-      block8<D>(s0 + SL::Q, s0 + SL::K + (j & 1) * SL::TILE16, s0 + SL::V + (j & 1) * SL::TILE16,
-                smem + SL::P + warp * 1024, region_mask(g, kb), sc, warp, lane, O, m, l, vs);
+      float ux0 = -INFINITY, ux1 = -INFINITY;
+      for (int t = 0; t < nm; ++t) {  // the unit's row maxima, scores only
+        float S[8][4], mx0, mx1;
+        qk_int8<D>(s0 + SL::Q, s0 + SL::K + t * SL::TILE16, warp, lane, S);
+        scale_mask(S, sq * A.k_s8[(size_t)bh * g.nb + kbs[t]] * sl2, region_mask(g, kbs[t]), tq, mx0, mx1);
+        ux0 = fmaxf(ux0, mx0); ux1 = fmaxf(ux1, mx1);
+      }
+      raise_ref(r, ux0, ux1);
+      for (int t = 0; t < nm; ++t) {
+        const float sc = sq * A.k_s8[(size_t)bh * g.nb + kbs[t]] * sl2;
+        block8<D>(s0 + SL::Q, s0 + SL::K + t * SL::TILE16, s0 + SL::V + t * SL::TILE16,
+                  smem + SL::P + warp * 1024, region_mask(g, kbs[t]), sc, warp, lane, O, m, l, vs, r);
+      }
       __syncthreads();
     }
   }
   // ---------------- phase 4
   if (cnt.z > 0) {
-    const uint16_t* l4 = list + cnt.x + cnt.y;
     dequant_f4_tile<D>(smem + SL::Q, A.q_f4 + row_lin * 64 * (D / 2), A.q_sf4 + row_lin * SL::KSF, 64);
     for (int c = threadIdx.x; c < D; c += kAttnThreads) vs[c] = A.v_g4[(size_t)bh * D + c];
-    auto issue = [&](int j) {
-      const size_t kl = (size_t)bh * g.nb + l4[j];
-      const uint32_t raw = s0 + SL::RAW + (j & 1) * SL::RAW_STAGE;
-      load_bytes(raw + SL::RAW_KC, A.k_f4 + kl * 64 * (D / 2), 64 * D / 2);
-      load_bytes(raw + SL::RAW_KS, A.k_sf4 + kl * SL::KSF, SL::KSF);
-      load_bytes(raw + SL::RAW_VC, A.v_f4 + kl * D * 32, D * 32);
-      load_bytes(raw + SL::RAW_VS, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes);
+    float r[2] = {-INFINITY, -INFINITY};
+    const uint32_t* it4 = items + pc.x + pc.y;
+    for (int i = 0; i < pc.z; i += 2) {
+      int kbs[2];
+      const int nm = unit_members(it4, pc.z, i, kbs);
+      if (nm == 0) continue;
+      for (int t = 0; t < nm; ++t) {
+        const size_t kl = (size_t)bh * g.nb + kbs[t];
+        const uint32_t raw = s0 + SL::RAW + t * SL::RAW_STAGE;
+        load_bytes(raw + SL::RAW_KC, A.k_f4 + kl * 64 * (D / 2), 64 * D / 2);
+        load_bytes(raw + SL::RAW_KS, A.k_sf4 + kl * SL::KSF, SL::KSF);
+        load_bytes(raw + SL::RAW_VC, A.v_f4 + kl * D * 32, D * 32);
+        load_bytes(raw + SL::RAW_VS, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes);
+      }
       cp_async_commit();
-    };
-    issue(0);
-    for (int j = 0; j < cnt.z; ++j) {
-      if (j + 1 < cnt.z) { issue(j + 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
+      cp_async_wait<0>();
       __syncthreads();
-      uint8_t* raw = smem + SL::RAW + (j & 1) * SL::RAW_STAGE;
-      uint8_t* kt = smem + SL::K + (j & 1) * SL::TILE16;
-      uint8_t* vt = smem + SL::V + (j & 1) * SL::TILE16;
-      dequant_f4_tile<D>(kt, raw + SL::RAW_KC, raw + SL::RAW_KS, 64);
-      dequant_f4_tile<64>(vt, raw + SL::RAW_VC, raw + SL::RAW_VS, D);
+      for (int t = 0; t < nm; ++t) {
+        uint8_t* raw = smem + SL::RAW + t * SL::RAW_STAGE;
+        dequant_f4_tile<D>(smem + SL::K + t * SL::TILE16, raw + SL::RAW_KC, raw + SL::RAW_KS, 64);
+        dequant_f4_tile<64>(smem + SL::V + t * SL::TILE16, raw + SL::RAW_VC, raw + SL::RAW_VS, D);
+      }
       __syncthreads();
-      block4<D>(s0 + SL::Q, smem_u32(kt), smem_u32(vt), region_mask(g, l4[j]), sl2, warp, lane, O, m, l, vs);
+      float ux0 = -INFINITY, ux1 = -INFINITY;
+      for (int t = 0; t < nm; ++t) {  // the unit's row maxima, scores only
+        float S[8][4], mx0, mx1;
+        qk_16bit<D, true>(s0 + SL::Q, s0 + SL::K + t * SL::TILE16, warp, lane, S);
+        scale_mask(S, sl2, region_mask(g, kbs[t]), tq, mx0, mx1);
+        ux0 = fmaxf(ux0, mx0); ux1 = fmaxf(ux1, mx1);
+      }
+      raise_ref(r, ux0, ux1);
+      for (int t = 0; t < nm; ++t)
+        block4<D>(s0 + SL::Q, s0 + SL::K + t * SL::TILE16, s0 + SL::V + t * SL::TILE16, region_mask(g, kbs[t]),
+                  sl2, warp, lane, O, m, l, vs, r);
       __syncthreads();
     }
   }
@@ -547,6 +609,8 @@ AttnArgs make_args(const Layout& L, const void* q, const void* k, const void* v,
   A.v_g4 = at<float>(ws, L, R_V_G4);
   A.lists = at<uint16_t>(ws, L, R_LISTS);
   A.counts = at<int>(ws, L, R_COUNTS);
+  A.plist = at<uint32_t>(ws, L, R_PLIST);
+  A.pcnt = at<int>(ws, L, R_PCNT);
   return A;
 }
 
@@ -556,6 +620,7 @@ cudaError_t launch_attention_d(const Geom& g, const Layout& L, const void* q, co
   const int smem = SmemLayout<D>::TOTAL;
   cudaError_t e = cudaFuncSetAttribute(attn_mp_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  if ((e = launch_pair_lists(g, L, ws, st)) != cudaSuccess) return e;
   attn_mp_kernel<D><<<dim3(g.nb, g.BH), kAttnThreads, smem, st>>>(g, make_args<D>(L, q, k, v, ws, out));
   return cudaGetLastError();
 }

@@ -15,28 +15,37 @@
 // and the other half's P rows are zero; on the video workloads 74-80 % of the
 // computed rows are useful, against 50 % for M = 64.
 //
-// Roles (10 warps): warps 0-7 softmax — warp w owns TMEM lanes 32(w&3).. (tile
-// rows) and half h = w>>2 of every key block (keys 32h..32h+31) and of the
-// channels (64h..64h+63); warp 8 issues TMA loads; warp 9 issues the MMAs from
-// a non-blocking scheduler that starts S of a block as soon as its buffers are
-// free, ahead of the P·V of the block before.
-//   16-bit  S = Q·K^T (kind::f16 bf16, M128 N64, fp32 TMEM, 2 buffers);
+// Units: every phase takes its key blocks two at a time (a, b).  Roles (10
+// warps): warps 0-7 softmax — warp w owns TMEM lanes 32(w&3).. (tile rows),
+// key block h = w>>2 of every unit (all 64 keys of it) and channels 64h..64h+63
+// of the output; warp 8 issues TMA loads; warp 9 issues the MMAs from a
+// non-blocking scheduler that starts S of a unit as soon as its buffers are
+// free, ahead of the P·V of the unit before.
+//   16-bit  S = Q·K^T (kind::f16 bf16, M128 N128, fp32 TMEM, 2 buffers);
 //           P = exp2(s·log2e/√d − m_ref) rounded to bf16, m_ref an integer
-//           exponent raised lazily (O rescaled in TMEM by a power of two only
-//           when the row max grows by more than 2^8); P goes K-major to shared
-//           memory; O += P·V (kind::f16, V read MN-major from the TMA tile).
-//   8-bit   S = Q8·K8^T (kind::i8, s32); P8 = round(255·exp(s − m_blk)) as u8;
-//           X = P8·V8^T (kind::i8 u8×s8, s32, 2 buffers); each softmax warp
-//           folds its 64 channels of X into a register accumulator weighted by
-//           exp(m_blk − m8); the per-channel V scale is applied once, at the
-//           phase boundary, when the register accumulator joins O.
-//   4-bit   S = Q4·K4^T (kind::mxf4nvf4, block16 e4m3 scales copied into TMEM
-//           with tcgen05.cp from the scale atoms prep wrote); P re-quantised to
-//           NVFP4 per 16 keys in registers, with its scales written as an atom;
-//           X = P4·V4^T (block-scaled, fp32), folded into the register
-//           accumulator; the channel scale g is applied at the end.  Entering
-//           the phase, the INT8 accumulator is folded into O with its own
-//           channel scale first — the phase-boundary rescale.
+//           exponent shared by the two warps of a row and raised lazily (O
+//           rescaled in TMEM by a power of two only when the row max grows by
+//           more than 2^8); P goes K-major to shared memory; O += P·V
+//           (kind::f16, V read MN-major from the TMA tile).
+//   Entering the low-bit phases, O moves into registers (each warp its 64
+//   channels), where it stays: the block results of the low-bit phases are
+//   folded into it, and TMEM holds one S buffer and the two block results.
+//   8-bit   S = Q8·[K8_a; K8_b]^T (kind::i8, s32, N128); each warp quantises its
+//           block's P8 = round(255·exp(s − m_blk)) as u8 from its own full
+//           rows, so no statistics cross warps before the MMA;
+//           X_h = P8_h·V8_h^T (kind::i8 u8×s8, s32).  Both warps of a row fold
+//           their 64 channels of X_a and X_b into the register accumulator with
+//           weight exp(m_blk − m); the two warps trade (m_blk, l_blk) through
+//           shared memory one unit late, off the critical path.
+//   4-bit   S_h = Q4·K4_h^T (kind::mxf4nvf4, block16 e4m3 scales copied into
+//           TMEM with tcgen05.cp from the scale atoms prep wrote); P
+//           re-quantised to NVFP4 per 16 keys in registers, with its scales
+//           written as an atom; X_h = P4_h·V4_h^T (block-scaled, fp32), folded
+//           in the same way.
+//   The register accumulator is kept divided by the channel scale of the
+//   phase it last took (INT8 sv, NVFP4 g), so a fold is one FMA per element;
+//   crossing a phase boundary re-expresses it in the next phase's scale, and
+//   the epilogue multiplies the last scale back.
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), INT8 codes as 2-D
 // boxes of the workspace.  The epilogue writes O through the same region box
@@ -62,42 +71,56 @@ constexpr int kThreads = 320;
 constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// INT8 MMAs accumulate onto the bit pattern of 1.5*2^23: an s32 result x
+// (|x| < 2^22) then reads as the float 1.5*2^23 + x, exact, and one
+// subtraction turns it into x.
+constexpr uint32_t kI8Bias = 0x4B400000u;
+constexpr float kI8BiasF = 12582912.0f;
+// the 4-bit phase quantises 2688 p: 6 (largest e2m1) x 448 (largest e4m3)
+constexpr float kP4Range = 2688.0f;
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q16 = 0;         // [2 halves][128 rows][128 B], SW128
 constexpr uint32_t SM_Q8 = 32768;      // [128 rows][128 B], SW128
 constexpr uint32_t SM_K = 49152;       // K ring: kStages x 32 KB
 constexpr uint32_t SM_V = SM_K + kStages * 32768;            // V ring: kStages x 32 KB
-// 16-bit unit (key blocks a, b): K slot = K_a h0 | K_b h0 | K_a h1 | K_b h1 (8 KB
-// each, so each channel half of [K_a; K_b] is one 128-row K-major operand);
-// V slot = V_a | V_b (16 KB each).  INT8 unit (one key block): K8 (8 KB), V8^T (8 KB).
-constexpr uint32_t SM_P = SM_V + kStages * 32768;            // P_a | P_b, 16 KB each
-constexpr uint32_t SM_VS = SM_P + 32768;                     // V channel scales: INT8 | NVFP4 g (fp32)
+// 16-bit unit: K slot = K_a h0 | K_b h0 | K_a h1 | K_b h1 (8 KB each, so each
+// channel half of [K_a; K_b] is one 128-row K-major operand); V slot = V_a | V_b
+// (16 KB each).  INT8 unit: K slot = K8_a | K8_b (8 KB each: one 128-row
+// operand), V slot = V8_a^T | V8_b^T (8 KB each).  4-bit unit: K slot =
+// K4_a | K4_b ([64][64 B] SW64, 4 KB each) with their scale atoms (2 x 512 B
+// per block) at +8192; V slot = V4_a^T | V4_b^T ([128][32 B] SW32, 4 KB each)
+// with one scale atom per block at +8192.
+constexpr uint32_t SL_SF = 8192;
+// P area: 16-bit P_a | P_b (16 KB each).  Low-bit units: P8_a | P8_b (8 KB
+// each) or P4_a | P4_b (4 KB each) at +0 and the P4 scale atoms at +16384.
+constexpr uint32_t SM_P = SM_V + kStages * 32768;
+constexpr uint32_t PO_PSF = 16384;
+// channel scales that fold a low-bit accumulator into O (fp32 [128] each):
+// INT8 sv/255 (P codes are 255 p) | NVFP4 g/2688 (P is quantised as 2688 p)
+constexpr uint32_t SM_VS = SM_P + 32768;
+constexpr uint32_t VS_SV255 = 0, VS_G2688 = 512;
 constexpr uint32_t SM_RED = SM_VS + 1024;                    // row-statistics exchange, 4 KB
 constexpr uint32_t SM_BAR = SM_RED + 4096;                   // mbarriers
 constexpr uint32_t SM_MISC = SM_BAR + 512;
-constexpr uint32_t SM_PSF = SM_MISC + 128;                   // scale atom of the 4-bit P (512 B)
-constexpr uint32_t SM_Q4 = (SM_PSF + 512 + 1023) & ~1023u;   // NVFP4 Q of the pair [128][64 B], SW64
+constexpr uint32_t SM_Q4 = (SM_MISC + 128 + 1023) & ~1023u;  // NVFP4 Q of the pair [128][64 B], SW64
 constexpr uint32_t SM_TOTAL = SM_Q4 + 8192;
-// 4-bit unit: K slot = K4 [64][64 B] SW64 at +0, its scale atoms (2 x 512 B) at
-// +8192; V slot = V4^T [128][32 B] SW32 at +0, its scale atom at +8192
-constexpr uint32_t SL_SF = 8192;
 constexpr uint32_t kSmemBytes = SM_TOTAL + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns: O 0-127, S 2 x 128 at 128 (a 16-bit unit fills 128, an INT8 or
-// 4-bit unit 64), X 128 at 384.  4-bit units keep their scale factors in the
-// upper half of their S buffer: K scales at +64, V scales at +72, P scales at
-// +76; Q's scales (constant for the CTA) at 216.  Scale columns are 4-aligned.
-constexpr uint32_t TM_O = 0, TM_S = 128, TM_X = 384;
-constexpr uint32_t TM_SFQ = 216, TMO_SFK = 64, TMO_SFV = 72, TMO_SFP = 76;
+// TMEM columns: O 0-127 (every phase); S 2 x 128 at 128 (16-bit and INT8
+// units; a 4-bit unit uses one, S_a 128 and S_b 192); the low-bit phase
+// accumulator at 384 (INT8 s32 X8, then 4-bit fp32 O4); 4-bit scale factors
+// from 256 — Q 256, K_a 264, K_b 272, V_a 280, V_b 284, P_a 288, P_b 292, all
+// 4-aligned as block-scaled MMAs require.
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_ACC = 384;
+constexpr uint32_t TM_SFQ = 256, TM_SFK = 264, TM_SFV = 280, TM_SFP = 288;
 
 // mbarrier slots (8 bytes each)
 enum {
   B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
   B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages,
-  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_X_FULL = B_P_FREE + 1,
-  B_X_FREE = B_X_FULL + 1, B_DONE = B_X_FREE + 1,
+  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_DONE = B_P_FREE + 1,
   B_PAIR = B_DONE + 1,   // [4 quarters][2 parities]: the two warps of a row quarter
   B_EPI = B_PAIR + 8,    // [4 quarters]: final exchange
   B_COUNT = B_EPI + 4
@@ -120,11 +143,6 @@ struct TcArgs {
 
 __device__ __forceinline__ void raise_timeout(int* status) { atomicOr(status, 1); }
 
-// Exact int32 -> fp32 for |x| < 2^22 on the integer and FMA pipes (the I2F
-// conversion unit is a narrow pipe): 1.5*2^23 + x has x in its low mantissa bits.
-__device__ __forceinline__ float i2f_small(uint32_t x) {
-  return __int_as_float((int)x + 0x4B400000) - 12582912.0f;
-}
 // packed fp32x2 arithmetic (one FMA-pipe instruction for two lanes' values)
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
   uint64_t r;
@@ -157,16 +175,10 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t x0, uint32_t x1, uin
   asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
   return r;
 }
-// round-to-nearest-even of a value in [0, 2^22) to an integer in the low bits,
-// again through the mantissa of 1.5*2^23 (the add rounds ties to even)
-__device__ __forceinline__ uint32_t rne_small(float v) {
-  return (uint32_t)__float_as_int(v + 12582912.0f) & 0x3FFFFFu;
-}
 
 // Items: kb | inA << 16 | inB << 17 | kind << 18 (kind 0 = 16-bit, 1 = 8-bit)
 //        | full << 20 (the key block has no padding slot).
 __device__ __forceinline__ int item_kb(uint32_t e) { return (int)(e & 0xffffu); }
-__device__ __forceinline__ int item_kind(uint32_t e) { return (int)((e >> 18) & 3u); }
 
 __device__ __forceinline__ bool item_full(uint32_t e) { return (e >> 20) & 1u; }
 
@@ -187,6 +199,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmV8, const __grid_constant__ CUtensorMap tmQ4,
                const __grid_constant__ CUtensorMap tmK4, const __grid_constant__ CUtensorMap tmV4, Geom g,
                TcArgs A) {
+  // a CTA that timed out raised the status word: later CTAs skip their work
+  if (*reinterpret_cast<volatile const int*>(A.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s0 = (uint32_t)__cvta_generic_to_shared(smem);
@@ -201,14 +215,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 8);
 
-  // units: 16-bit items are taken two at a time (one N = 128 score MMA per
-  // unit), INT8 items one at a time
+  // units: each phase takes its items (key blocks) two at a time, in list order
   const int nu16 = (n16 + 1) / 2;
-  const int nu8 = nu16 + n8;  // INT8 units end here, 4-bit units follow
-  const int nu = nu8 + n4;
+  const int nu8 = nu16 + (n8 + 1) / 2;  // INT8 units end here, 4-bit units follow
+  const int nu = nu8 + (n4 + 1) / 2;
   auto unit_items = [&](int u, int& i0, int& cnt) {
-    if (u < nu16) { i0 = 2 * u; cnt = min(2, n16 - 2 * u); }
-    else { i0 = n16 + (u - nu16); cnt = 1; }  // INT8 and 4-bit items follow in list order
+    if (u < nu16) { i0 = 2 * u; cnt = min(2, n16 - i0); }
+    else if (u < nu8) { i0 = n16 + 2 * (u - nu16); cnt = min(2, n16 + n8 - i0); }
+    else { i0 = n16 + n8 + 2 * (u - nu8); cnt = min(2, n16 + n8 + n4 - i0); }
   };
 
   if (threadIdx.x == 0) {
@@ -226,8 +240,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     mbar_init(bar(B_P_FULL), kSoftmaxWarps);
     mbar_init(bar(B_P_FREE), 1);
-    mbar_init(bar(B_X_FULL), 1);
-    mbar_init(bar(B_X_FREE), kSoftmaxWarps);
     mbar_init(bar(B_DONE), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(B_PAIR + i), 2);
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_EPI + i), 2);
@@ -236,13 +248,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   if (warp == kMmaWarp) tmem_alloc(s0 + SM_MISC, 512);
   if (threadIdx.x < kD) {
-    reinterpret_cast<float*>(smem + SM_VS)[threadIdx.x] = A.v_s8[(size_t)bh * kD + threadIdx.x];
-    reinterpret_cast<float*>(smem + SM_VS + 512)[threadIdx.x] = A.v_g4[(size_t)bh * kD + threadIdx.x];
+    const float sv = A.v_s8[(size_t)bh * kD + threadIdx.x], gv = A.v_g4[(size_t)bh * kD + threadIdx.x];
+    float* vsc = reinterpret_cast<float*>(smem + SM_VS);
+    vsc[VS_SV255 / 4 + threadIdx.x] = sv / 255.0f;
+    vsc[VS_G2688 / 4 + threadIdx.x] = gv / kP4Range;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = misc[0];
+  if (warp < kSoftmaxWarps) {
+    // S buffers whose first user is an INT8 unit start at the bias
+    const uint32_t own = tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * 64;
+    bool any = false;
+    if (n8 > 0 || n4 > 0) {  // the low-bit accumulator starts at zero
+      tmem_fill32(own + TM_ACC, 0u);
+      tmem_fill32(own + TM_ACC + 32, 0u);
+      any = true;
+    }
+    for (int b = 0; b < 2; ++b)
+      if (b >= nu16 && b < nu8) {
+        tmem_fill32(own + TM_S + b * 128, kI8Bias);
+        tmem_fill32(own + TM_S + b * 128 + 32, kI8Bias);
+        any = true;
+      }
+    if (any) tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   const int t_of = g.nry * g.nrx;  // blocks per frame
   auto box = [&](int blk, int& cx, int& cy, int& cf) {
@@ -296,13 +330,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_4d(dst + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
             }
           } else if (kn < nu8) {
-            mbar_expect_tx(fb, 8192u);
-            tma_load_2d(dst, &tmK8, fb, 0, (bh * g.nb + item_kb(items[i0])) * 64);
+            mbar_expect_tx(fb, 8192u * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t)
+              tma_load_2d(dst + t * 8192, &tmK8, fb, 0, (bh * g.nb + item_kb(items[i0 + t])) * 64);
           } else {
-            const size_t kl = (size_t)bh * g.nb + item_kb(items[i0]);
-            mbar_expect_tx(fb, 4096u + 1024u);
-            tma_load_2d(dst, &tmK4, fb, 0, (int)(kl * 64));
-            bulk_load(dst + SL_SF, A.k_sf4 + kl * 2 * kSfAtomBytes, 2 * kSfAtomBytes, fb);
+            mbar_expect_tx(fb, (4096u + 2 * kSfAtomBytes) * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t) {
+              const size_t kl = (size_t)bh * g.nb + item_kb(items[i0 + t]);
+              tma_load_2d(dst + t * 4096, &tmK4, fb, 0, (int)(kl * 64));
+              bulk_load(dst + SL_SF + t * 2 * kSfAtomBytes, A.k_sf4 + kl * 2 * kSfAtomBytes, 2 * kSfAtomBytes, fb);
+            }
           }
           ++kn;
           progressed = true;
@@ -320,22 +357,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               tma_load_4d(dst + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
             }
           } else if (vn < nu8) {
-            mbar_expect_tx(fb, 8192u);
-            tma_load_2d(dst, &tmV8, fb, 0, (bh * g.nb + item_kb(items[i0])) * kD);
+            mbar_expect_tx(fb, 8192u * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t)
+              tma_load_2d(dst + t * 8192, &tmV8, fb, 0, (bh * g.nb + item_kb(items[i0 + t])) * kD);
           } else {
-            const size_t kl = (size_t)bh * g.nb + item_kb(items[i0]);
-            mbar_expect_tx(fb, 4096u + kSfAtomBytes);
-            tma_load_2d(dst, &tmV4, fb, 0, (int)(kl * kD));
-            bulk_load(dst + SL_SF, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
+            mbar_expect_tx(fb, (4096u + kSfAtomBytes) * (uint32_t)cnt);
+            for (int t = 0; t < cnt; ++t) {
+              const size_t kl = (size_t)bh * g.nb + item_kb(items[i0 + t]);
+              tma_load_2d(dst + t * 4096, &tmV4, fb, 0, (int)(kl * kD));
+              bulk_load(dst + SL_SF + t * kSfAtomBytes, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
+            }
           }
           ++vn;
           progressed = true;
         }
         if (progressed) {
           idle = 0;
-        } else if (++idle > (1u << 26) || *abort_flag) {
+        } else if (++idle > (1u << 24) || *abort_flag) {
           raise_timeout(A.status); *abort_flag = 1;
           break;
+        } else {
+          __nanosleep(64);  // leave the issue slots of this sub-partition to the softmax warps
         }
       }
     }
@@ -345,31 +387,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t id16n128 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 128);
       const uint32_t id16n64 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 64);
       const uint32_t idpv = idesc(kDF32, kFmtBF16, kFmtBF16, false, true, 128, 128);
-      const uint32_t id8 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
+      const uint32_t id8n64 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
+      const uint32_t id8n128 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 128);
       const uint32_t idx8 = idesc(kDS32, kFmtU8, kFmtS8, false, false, 128, 128);
       const uint32_t id4s = idesc_f4(128, 64), id4pv = idesc_f4(128, 128);
       bool f4_ready = false;  // Q4 loaded and its scales in TMEM
       bool ok = true;
       if (n16 > 0) ok = ok && mbar_wait(bar(B_Q16), 0);
       if (n8 > 0) ok = ok && mbar_wait(bar(B_Q8), 0);
-      int sn = 0, pn = 0, xu = 0;  // next unit for S, next unit for P·V, INT8 results issued
+      int sn = 0, pn = 0;  // next unit for S, next unit for P·V
       uint32_t idle = 0;
       while (ok && pn < nu) {
         bool progressed = false;
         if (sn < nu) {
           const int s = sn % kStages, b = sn & 1;
-          if (sn >= nu8 && !f4_ready) {
+          const bool single = sn >= nu8;
+          if (single && !f4_ready) {
             // first 4-bit unit: Q4 must be in shared memory and its scales in TMEM
             f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
           }
-          if ((sn < nu8 || f4_ready) && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1) &&
-              (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1))) {
+          // 16-bit and INT8 units alternate two S buffers; 4-bit units share
+          // one (the second holds scale factors), so they wait for the unit
+          // before — for the first of them that implies both buffers were read
+          const bool s_free = single ? (sn < 1 || mbar_test(bar(B_S_FREE + ((sn - 1) & 1)), ((sn - 1) >> 1) & 1))
+                                     : (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1));
+          if ((sn < nu8 || f4_ready) && s_free && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1)) {
             tc_fence_after();
             const uint32_t st = s0 + SM_K + s * 32768;
-            const uint32_t sd = tbase + TM_S + b * 128;
+            const uint32_t sd = tbase + TM_S + (single ? 0u : b * 128u);
+            int i0, cnt;
+            unit_items(sn, i0, cnt);
             if (sn < nu16) {
-              int i0, cnt;
-              unit_items(sn, i0, cnt);
               const uint32_t id = cnt == 2 ? id16n128 : id16n64;
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
@@ -378,16 +426,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         smem_desc(st + h * 16384 + kk * 32, 16, 1024, SW_128), id, k > 0 ? 1u : 0u);
               }
             } else if (sn < nu8) {
+              const uint32_t id = cnt == 2 ? id8n128 : id8n64;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
-                       smem_desc(st + kk * 32, 16, 1024, SW_128), id8, kk > 0 ? 1u : 0u);
+                       smem_desc(st + kk * 32, 16, 1024, SW_128), id, 1u);  // onto the bias
             } else {
+              for (int t = 0; t < cnt; ++t) {
+                const uint32_t sfk = tbase + TM_SFK + 8 * t;
 #pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                tc_cp_atom(sd + TMO_SFK + 4 * c, st + SL_SF + c * kSfAtomBytes);
-                mma_f4(sd, smem_desc(s0 + SM_Q4 + 32 * c, 16, 512, SW_64), smem_desc(st + 32 * c, 16, 512, SW_64),
-                       id4s, c > 0 ? 1u : 0u, tbase + TM_SFQ + 4 * c, sd + TMO_SFK + 4 * c);
+                for (int c = 0; c < 2; ++c) {
+                  tc_cp_atom(sfk + 4 * c, st + SL_SF + (2 * t + c) * kSfAtomBytes);
+                  mma_f4(sd + 64 * t, smem_desc(s0 + SM_Q4 + 32 * c, 16, 512, SW_64),
+                         smem_desc(st + t * 4096 + 32 * c, 16, 512, SW_64), id4s, c > 0 ? 1u : 0u,
+                         tbase + TM_SFQ + 4 * c, sfk + 4 * c);
+                }
               }
             }
             mma_commit(bar(B_S_FULL + b));
@@ -398,13 +451,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (pn < sn) {
           const int s = pn % kStages;
-          const bool int8 = pn >= nu16;  // INT8 or 4-bit: both produce a block result X
-          if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL), pn & 1) &&
-              (!int8 || xu < 1 || mbar_test(bar(B_X_FREE), (xu - 1) & 1))) {
+          const bool low = pn >= nu16;  // INT8 or 4-bit: P·V accumulates at TM_ACC
+          // (the softmax warps settle the accumulator before they release P)
+          if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL), pn & 1)) {
             tc_fence_after();
             const uint32_t st = s0 + SM_V + s * 32768;
             const uint32_t pbuf = s0 + SM_P;
-            if (!int8) {
+            if (!low) {
               int i0, cnt;
               unit_items(pn, i0, cnt);
               for (int t = 0; t < cnt; ++t) {
@@ -414,20 +467,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                           smem_desc(st + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
               }
             } else if (pn < nu8) {
+              int i0, cnt;
+              unit_items(pn, i0, cnt);
+              for (int t = 0; t < cnt; ++t) {
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk)
-                mma_i8(tbase + TM_X, smem_desc(pbuf + kk * 32, 16, 512, SW_64),
-                       smem_desc(st + kk * 32, 16, 512, SW_64), idx8, kk > 0 ? 1u : 0u);
-              mma_commit(bar(B_X_FULL));
-              ++xu;
+                for (int kk = 0; kk < 2; ++kk)
+                  mma_i8(tbase + TM_ACC, smem_desc(pbuf + t * 8192 + kk * 32, 16, 512, SW_64),
+                         smem_desc(st + t * 8192 + kk * 32, 16, 512, SW_64), idx8, 1u);
+              }
             } else {
-              const uint32_t sfb = tbase + TM_S + (pn & 1) * 128;
-              tc_cp_atom(sfb + TMO_SFV, st + SL_SF);
-              tc_cp_atom(sfb + TMO_SFP, s0 + SM_PSF);
-              mma_f4(tbase + TM_X, smem_desc(pbuf, 16, 256, SW_32), smem_desc(st, 16, 256, SW_32), id4pv, 0u,
-                     sfb + TMO_SFP, sfb + TMO_SFV);
-              mma_commit(bar(B_X_FULL));
-              ++xu;
+              int i0, cnt;
+              unit_items(pn, i0, cnt);
+              for (int t = 0; t < cnt; ++t) {
+                const uint32_t sfv = tbase + TM_SFV + 4 * t, sfp = tbase + TM_SFP + 4 * t;
+                tc_cp_atom(sfv, st + SL_SF + t * kSfAtomBytes);
+                tc_cp_atom(sfp, pbuf + PO_PSF + t * kSfAtomBytes);
+                mma_f4(tbase + TM_ACC, smem_desc(pbuf + t * 4096, 16, 256, SW_32),
+                       smem_desc(st + t * 4096, 16, 256, SW_32), id4pv, 1u, sfp, sfv);
+              }
             }
             mma_commit(bar(B_P_FREE));
             mma_commit(bar(B_V_EMPTY + s));
@@ -437,8 +494,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (progressed) {
           idle = 0;
-        } else if (++idle > (1u << 26) || *abort_flag) {
+        } else if (++idle > (1u << 24) || *abort_flag) {
           ok = false;
+        } else {
+          __nanosleep(32);  // leave the issue slots of this sub-partition to the softmax warps
         }
       }
       mma_commit(bar(B_DONE));
@@ -453,7 +512,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = kLog2e * rsqrtf((float)kD);
     const float sq = (n8 > 0 && qrow_blk >= 0) ? A.q_s8[(size_t)bh * g.nb + qrow_blk] : 0.f;
-    const float* vs = reinterpret_cast<const float*>(smem + SM_VS);
     float* red = reinterpret_cast<float*>(smem + SM_RED);  // [2][2][128]
     const unsigned FULL = 0xffffffffu;
     // the two warps of a row quarter exchange row statistics through shared
@@ -464,7 +522,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return __all_sync(FULL, mbar_wait(bar(idx), parity));
     };
     float m16 = -INFINITY, l16 = 0.f;  // 16-bit phase: O in TMEM, integer reference
-    float m8 = -INFINITY, l8 = 0.f;    // 8-bit phase: register accumulator
     bool ok = true;
     {  // O starts at zero (this warp's 64 columns)
       uint32_t z[32];
@@ -492,6 +549,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tmem_ld32(sbase + half * 64, sr);
           tmem_ld32(sbase + half * 64 + 32, sr + 32);
           tmem_wait_ld();
+        }
+        if (u + 2 >= nu16 && u + 2 < nu8) {  // the buffer's next user is an INT8 unit
+          tmem_fill32(sbase + half * 64, kI8Bias);
+          tmem_fill32(sbase + half * 64 + 32, kI8Bias);
+          tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
@@ -570,175 +632,73 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_P_FULL));
     }
-    // the INT8 register accumulator lives only through the 8-bit phase
-    float o8[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) o8[i] = 0.f;
-    int xu = 0;
-    bool have_pend = false, pend_member = false;
-    float pend_mb = 0.f, pend_lb = 0.f;
-    // fold the X of the pending INT8 item into the register accumulator
-    auto merge_x = [&]() -> bool {
-      if (!__all_sync(FULL, mbar_wait(bar(B_X_FULL), xu & 1))) return false;
-      tc_fence_after();
-      if (pend_member) {
-        uint32_t xr[64];
-        tmem_ld32(tbase + lane_off + TM_X + half * 64, xr);
-        tmem_ld32(tbase + lane_off + TM_X + half * 64 + 32, xr + 32);
-        tmem_wait_ld();
-        if (pend_mb > m8 + kRescaleThreshold || m8 == -INFINITY) {
-          const float nm = ceilf(pend_mb);
-          const float a = (m8 == -INFINITY) ? 0.f : ldexpf(1.0f, (int)(m8 - nm));
-#pragma unroll
-          for (int i = 0; i < 64; ++i) o8[i] *= a;
-          l8 *= a;
-          m8 = nm;
-        }
-        const float w = fast_exp2(pend_mb - m8);
-        const float f = w * (1.0f / 255.0f);
-        l8 += pend_lb * w;
-        const uint64_t fx2 = f2pack(f, f), kx2 = f2pack(-12582912.0f, -12582912.0f);
-#pragma unroll
-        for (int i = 0; i < 64; i += 2) {  // |X| < 64*255*127 < 2^22: exact through the mantissa
-          const uint64_t xf = f2add(f2pack(__int_as_float((int)xr[i] + 0x4B400000),
-                                           __int_as_float((int)xr[i + 1] + 0x4B400000)), kx2);
-          f2unpack(f2fma(fx2, xf, f2pack(o8[i], o8[i + 1])), o8[i], o8[i + 1]);
-        }
+    // ================================================================ low-bit phases
+    // Each low-bit phase accumulates P·V in TMEM (INT8: s32 X8; 4-bit: fp32
+    // O4, both at column 384) against its own power-of-two reference r per
+    // row, shared by the two warps of the row; P is quantised relative to 2^r.
+    // When a unit's row maximum exceeds r, the accumulator is first folded
+    // into O with the phase's channel scale (sv/255 or g/2688) and cleared;
+    // so is it at the end of the phase.  l8/l4 are this warp's partial sums
+    // against the same reference.
+    const float* chs8 = reinterpret_cast<const float*>(smem + SM_VS + VS_SV255);
+    const float* chs4 = reinterpret_cast<const float*>(smem + SM_VS + VS_G2688);
+    float r_lo = -INFINITY, l_lo = 0.f;
+    // fold the phase accumulator (this warp's 64 channels) into O for the
+    // lanes in `sel`; O's reference becomes max(m16, r_lo) for them
+    auto fold = [&](bool sel, bool i8) {
+      if (!__any_sync(FULL, sel)) return;
+      float a16 = 1.f, ax = 0.f;
+      if (sel && r_lo != -INFINITY) {
+        const float R = fmaxf(m16, r_lo);
+        a16 = m16 == -INFINITY ? 0.f : ldexpf(1.0f, (int)(m16 - R));
+        ax = ldexpf(1.0f, (int)(r_lo - R));
+        l16 = l16 * a16 + l_lo * ax;
+        m16 = R;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_X_FREE));
-      ++xu;
-      have_pend = false;
-      return true;
+      if (sel) l_lo = 0.f;
+      const float* chs = (i8 ? chs8 : chs4) + half * 64;
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 16) {
+        uint32_t orr[16], xr[16];
+        tmem_ld16(tbase + lane_off + TM_O + half * 64 + c, orr);
+        tmem_ld16(tbase + lane_off + TM_ACC + half * 64 + c, xr);
+        tmem_wait_ld();
+        if (sel) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x = i8 ? __int2float_rn((int)xr[i]) : __uint_as_float(xr[i]);
+            orr[i] = __float_as_uint(fmaf(x, ax * chs[c + i], __uint_as_float(orr[i]) * a16));
+            xr[i] = 0u;  // s32 0 and fp32 +0 alike
+          }
+        }
+        tmem_st16(tbase + lane_off + TM_O + half * 64 + c, orr);
+        tmem_st16(tbase + lane_off + TM_ACC + half * 64 + c, xr);
+      }
+      tmem_wait_st();
     };
-
-    for (int u = nu16; ok && u < nu8; ++u) {
+    for (int u = nu16; ok && u < nu; ++u) {
       if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-      const int b = u & 1;
+      const bool i8 = u < nu8;
+      if (u == nu8 && nu8 > nu16) {
+        // INT8 -> 4-bit boundary: the INT8 accumulator joins O once its last
+        // P·V completed; the columns then start the 4-bit accumulator at zero
+        if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        fold(true, true);
+        r_lo = -INFINITY;
+      }
       int i0, cnt;
       unit_items(u, i0, cnt);
-      float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
-      const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
-      // ---- INT8 unit: one key block; this warp owns keys 32*half..+31
-      const uint32_t e = items[i0];
+      // ---- this warp's block of the unit: key block `half`, all 64 keys
+      const bool present = half < cnt;
+      const uint32_t e = present ? items[i0 + half] : 0u;
       const int kb = item_kb(e);
-      const float sk = A.k_s8[(size_t)bh * g.nb + kb];  // issued before the wait
-      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
-      tc_fence_after();
-        const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
-        uint32_t sr[32];
-        tmem_ld32(sbase + half * 32, sr);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
-        const unsigned long long vm = item_full(e) ? ~0ull : (key_mask(g, kb) >> (32 * half));
-        const bool full = (uint32_t)vm == 0xffffffffu;
-        int imx = INT_MIN;
-        if (member) {
-          if (!full) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (!((vm >> i) & 1ull)) sr[i] = (uint32_t)INT_MIN;
-          }
-          int i4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) i4[i & 3] = max(i4[i & 3], (int)sr[i]);
-          imx = max(max(i4[0], i4[1]), max(i4[2], i4[3]));
-        }
-        reinterpret_cast<int*>(xch)[half * 128 + row] = imx;
-        if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
-        imx = max(imx, reinterpret_cast<const int*>(xch)[(1 - half) * 128 + row]);
-        float mb = -INFINITY, lb = 0.f;
-        uint32_t pw[8];
-        if (member) {
-          const float sc = sq * sk * sl2;
-          mb = i2f_small((uint32_t)imx) * sc;  // sc >= 0: the max of the scores; |S| < 128*127^2 < 2^22
-          const uint64_t scx2 = f2pack(sc, sc), negm = f2pack(-mb, -mb);
-          const uint64_t kx2 = f2pack(-12582912.0f, -12582912.0f);
-          const uint64_t c255 = f2pack(255.0f, 255.0f), kmag = f2pack(12582912.0f, 12582912.0f);
-          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint32_t c[4];
-#pragma unroll
-            for (int q = 0; q < 4; q += 2) {
-              const int k = 4 * i + q;
-              // exact int -> float through the mantissa of 1.5*2^23, then the score
-              const uint64_t sf = f2add(f2pack(__int_as_float((int)sr[k] + 0x4B400000),
-                                               __int_as_float((int)sr[k + 1] + 0x4B400000)), kx2);
-              float x0, x1;
-              f2unpack(f2fma(sf, scx2, negm), x0, x1);
-              float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              if (!full) {  // padding keys contribute nothing, whatever the block scale
-                if (!((vm >> k) & 1ull)) p0 = 0.f;
-                if (!((vm >> (k + 1)) & 1ull)) p1 = 0.f;
-              }
-              const uint64_t pp = f2pack(p0, p1);
-              acc[(i * 2 + (q >> 1)) & 3] = f2add(acc[(i * 2 + (q >> 1)) & 3], pp);
-              float r0, r1;  // 255 p + 1.5*2^23: round-to-nearest-even code in the low byte
-              f2unpack(f2fma(pp, c255, kmag), r0, r1);
-              c[q] = __float_as_uint(r0);
-              c[q + 1] = __float_as_uint(r1);
-            }
-            pw[i] = pack_low_bytes(c[0], c[1], c[2], c[3]);
-          }
-          float s0, s1, s2, s3;
-          f2unpack(f2add(acc[0], acc[1]), s0, s1);
-          f2unpack(f2add(acc[2], acc[3]), s2, s3);
-          lb = (s0 + s1) + (s2 + s3);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pw[i] = 0u;
-        }
-        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
-        uint8_t* pb = smem + SM_P;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int chunk = half * 2 + c;
-          *reinterpret_cast<uint4*>(pb + row * 64 + ((chunk ^ ((row >> 1) & 3)) * 16)) =
-              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_P_FULL));
-        if (have_pend && !merge_x()) { ok = false; break; }
-        have_pend = true;
-        pend_member = member;
-        pend_mb = mb;
-        pend_lb = lb;
-    }
-    if (ok && have_pend) ok = merge_x();
-    const float* vsc = reinterpret_cast<const float*>(smem + SM_VS);  // scale of the register accumulator
-    if (ok && n4 > 0) {
-      // ---- phase boundary 8 -> 4: fold the INT8 accumulator into O with its
-      // channel scale, so the registers can carry the 4-bit phase
-      if (n8 > 0) {
-        const float mm = fmaxf(m16, m8);
-        const float a16 = m16 == -INFINITY ? 0.f : fast_exp2(m16 - mm);
-        const float a8 = m8 == -INFINITY ? 0.f : fast_exp2(m8 - mm);
-#pragma unroll
-        for (int c = 0; c < 64; c += 32) {
-          uint32_t orr[32];
-          tmem_ld32(tbase + lane_off + TM_O + half * 64 + c, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            orr[i] = __float_as_uint(a16 * __uint_as_float(orr[i]) + a8 * vs[half * 64 + c + i] * o8[c + i]);
-          tmem_st32(tbase + lane_off + TM_O + half * 64 + c, orr);
-        }
-        tmem_wait_st();
-        l16 = l16 * a16 + l8 * a8;
-        m16 = mm;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) o8[i] = 0.f;
-        m8 = -INFINITY;
-        l8 = 0.f;
-      }
-      // Q's scale factors into TMEM (each lane quarter holds all 128 rows)
-      if (half == 0) {
+      const bool member = present && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
+      const float sk = (i8 && present) ? A.k_s8[(size_t)bh * g.nb + kb] : 0.f;  // issued before the wait
+      if (u == nu8 && half == 0) {
+        // first 4-bit unit: Q's scale factors into TMEM (each lane quarter
+        // holds all 128 rows).  The columns were the second S buffer, whose
+        // scores this warp has read, and no S MMA writes there any more.
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t w[4];
@@ -759,150 +719,182 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_SFQ));
       }
-      vsc = reinterpret_cast<const float*>(smem + SM_VS + 512);  // g
-      // fold a 4-bit block result X (fp32) into the register accumulator
-      auto merge_x4 = [&]() -> bool {
-        if (!__all_sync(FULL, mbar_wait(bar(B_X_FULL), xu & 1))) return false;
-        tc_fence_after();
-        if (pend_member) {
-          uint32_t xr[64];
-          tmem_ld32(tbase + lane_off + TM_X + half * 64, xr);
-          tmem_ld32(tbase + lane_off + TM_X + half * 64 + 32, xr + 32);
-          tmem_wait_ld();
-          if (pend_mb > m8 + kRescaleThreshold || m8 == -INFINITY) {
-            const float nm = ceilf(pend_mb);
-            const float a = (m8 == -INFINITY) ? 0.f : ldexpf(1.0f, (int)(m8 - nm));
-#pragma unroll
-            for (int i = 0; i < 64; ++i) o8[i] *= a;
-            l8 *= a;
-            m8 = nm;
-          }
-          const float f = fast_exp2(pend_mb - m8);
-          l8 += pend_lb * f;
-          const uint64_t fx2 = f2pack(f, f);
-#pragma unroll
-          for (int i = 0; i < 64; i += 2)
-            f2unpack(f2fma(fx2, f2pack(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), f2pack(o8[i], o8[i + 1])),
-                     o8[i], o8[i + 1]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_X_FREE));
-        ++xu;
-        have_pend = false;
-        return true;
-      };
-      for (int u = nu8; ok && u < nu; ++u) {
-        if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-        const int b = u & 1;
-        int i0, cnt;
-        unit_items(u, i0, cnt);
-        float* xch = red + (u & 1) * 256;
-        const uint32_t sbase = tbase + lane_off + TM_S + b * 128;
-        // ---- 4-bit unit: one key block; this warp owns keys 32*half..+31
-        const uint32_t e = items[i0];
-        const int kb = item_kb(e);
-        const bool member = ((e >> (in_b ? 17 : 16)) & 1u) != 0;
-        if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + b), (u >> 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld32(sbase + half * 32, sr);
+      float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
+      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      // this warp's scores: 64 columns of the unit's S buffer
+      const uint32_t scol = tbase + lane_off + TM_S + (i8 ? (uint32_t)(u & 1) * 128u : 0u) + half * 64;
+      const unsigned long long vm = item_full(e) ? ~0ull : key_mask(g, kb);
+      const bool full = vm == ~0ull;
+      uint32_t sr[64];
+      float mx = -INFINITY;
+      const float sc = i8 ? sq * sk * sl2 : sl2;  // score scale, log2 units (INT8: >= 0)
+      // member is uniform across the warp (its rows belong to one query block)
+      if (member) {
+        tmem_ld32(scol, sr);
+        tmem_ld32(scol + 32, sr + 32);
         tmem_wait_ld();
+        if (i8) {
+          // the s32 scores sit on the bias: subtracting it gives them exactly (|S| < 128*127^2 < 2^22)
+          const uint64_t kx2 = f2pack(-kI8BiasF, -kI8BiasF);
+#pragma unroll
+          for (int i = 0; i < 64; i += 2) {
+            float a, b;
+            f2unpack(f2add(f2pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), kx2), a, b);
+            sr[i] = __float_as_uint(a);
+            sr[i + 1] = __float_as_uint(b);
+          }
+        }
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
+        }
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; i += 8)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
+        mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sc;
+      }
+      if (!i8) {  // 4-bit units share one S buffer: release it at once
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + b));
-        const unsigned long long vm = item_full(e) ? ~0ull : (key_mask(g, kb) >> (32 * half));
-        const bool full = (uint32_t)vm == 0xffffffffu;
-        float mx = -INFINITY;
-        if (member) {
-          if (!full) {
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + (u & 1)));
+      }
+      xch[half * 128 + row] = mx;
+      if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+      mx = fmaxf(mx, xch[(1 - half) * 128 + row]);  // the unit's row maximum
+      // the reference rises to ceil(max) whenever the max exceeds it
+      const bool raise = mx != -INFINITY && (r_lo == -INFINITY || mx > r_lo);
+      const float r_use = raise ? ceilf(mx) : r_lo;
+      float lp = 0.f;  // this warp's sum of the unquantised p of the unit
+      uint32_t pw[16];
+      uint32_t sfw = 0u;  // 4-bit: the row's four e4m3 P scales
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
+      for (int i = 0; i < 16; ++i) pw[i] = 0u;
+      if (member) {
+        const uint64_t scx2 = f2pack(sc, sc), negr = f2pack(-r_use, -r_use);
+        uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
+        // p = exp2(s*sc - r) in place of the scores
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float x0, x1;
+          f2unpack(f2fma(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), scx2, negr), x0, x1);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (!full) {  // padding keys contribute nothing, whatever the block scale (sc may be 0)
+            if (!((vm >> (2 * i)) & 1ull)) p0 = 0.f;
+            if (!((vm >> (2 * i + 1)) & 1ull)) p1 = 0.f;
           }
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int i = 0; i < 32; i += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
-          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+          ls[i & 3] = f2add(ls[i & 3], f2pack(p0, p1));
+          sr[2 * i] = __float_as_uint(p0);
+          sr[2 * i + 1] = __float_as_uint(p1);
         }
-        xch[half * 128 + row] = mx;
-        if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
-        mx = fmaxf(mx, xch[(1 - half) * 128 + row]);
-        float mb = -INFINITY, lb = 0.f;
-        uint32_t pw[4] = {0u, 0u, 0u, 0u};
-        uint32_t sfw = 0u;  // this half-row's two e4m3 P scales
-        if (member) {
-          mb = mx * sl2;
-          float pv[32];
-          const uint64_t sl2x2 = f2pack(sl2, sl2), negm = f2pack(-mb, -mb);
+        float s0, s1, s2, s3;
+        f2unpack(f2add(ls[0], ls[1]), s0, s1);
+        f2unpack(f2add(ls[2], ls[3]), s2, s3);
+        lp = (s0 + s1) + (s2 + s3);
+        if (i8) {
+          const uint64_t c255 = f2pack(255.0f, 255.0f), kmag = f2pack(12582912.0f, 12582912.0f);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            f2unpack(f2fma(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm), x0, x1);
-            pv[2 * i] = fast_exp2(x0);
-            pv[2 * i + 1] = fast_exp2(x1);
+            uint32_t c[4];
+#pragma unroll
+            for (int q = 0; q < 4; q += 2) {
+              float r0, r1;  // 255 p + 1.5*2^23: round-to-nearest-even code in the low byte
+              f2unpack(f2fma(f2pack(__uint_as_float(sr[4 * i + q]), __uint_as_float(sr[4 * i + q + 1])), c255, kmag),
+                       r0, r1);
+              c[q] = __float_as_uint(r0);
+              c[q + 1] = __float_as_uint(r1);
+            }
+            pw[i] = pack_low_bytes(c[0], c[1], c[2], c[3]);
           }
+        } else {
+          // NVFP4 of 2688 p over 16 consecutive keys: e4m3 scale from the microblock max / 6
 #pragma unroll
-          for (int i = 0; i < 32; ++i) lb += pv[i];
-          // NVFP4 over 16 consecutive keys: e4m3 scale from the microblock max / 6
-#pragma unroll
-          for (int mbk = 0; mbk < 2; ++mbk) {
+          for (int mbk = 0; mbk < 4; ++mbk) {
             float pm = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pm = fmaxf(pm, pv[16 * mbk + i]);
-            const uint32_t sf = cvt_e4m3x2(0.0f, __fdiv_rn(pm, 6.0f)) & 0xffu;
+            for (int i = 0; i < 16; i += 2)
+              pm = fmax3(pm, __uint_as_float(sr[16 * mbk + i]), __uint_as_float(sr[16 * mbk + i + 1]));
+            const uint32_t sf = cvt_e4m3x2(0.0f, (pm * kP4Range) * (1.0f / 6.0f)) & 0xffu;
             sfw |= sf << (8 * mbk);
             const float dec = e4m3_to_f32(sf);
-            if (dec != 0.f) {
-              const float r = __fdiv_rn(1.0f, dec);
+            const float rr = dec != 0.f ? kP4Range * __frcp_rn(dec) : 0.f;
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                uint32_t w = 0;
+            for (int q = 0; q < 2; ++q) {
+              uint32_t w = 0;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  const int k = 16 * mbk + 8 * q + 2 * t;
-                  w |= cvt_e2m1x2(__fmul_rn(pv[k + 1], r), __fmul_rn(pv[k], r)) << (8 * t);
-                }
-                pw[2 * mbk + q] = w;
+              for (int t = 0; t < 4; ++t) {
+                const int k = 16 * mbk + 8 * q + 2 * t;
+                w |= cvt_e2m1x2(__uint_as_float(sr[k + 1]) * rr, __uint_as_float(sr[k]) * rr) << (8 * t);
               }
+              pw[2 * mbk + q] = w;
             }
           }
         }
-        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
-        *reinterpret_cast<uint4*>(smem + SM_P + row * 32 + ((half ^ ((row >> 2) & 1)) * 16)) =
-            make_uint4(pw[0], pw[1], pw[2], pw[3]);
-        *reinterpret_cast<uint16_t*>(smem + SM_PSF + (row & 31) * 16 + (row >> 5) * 4 + 2 * half) = (uint16_t)sfw;
-        fence_async_smem();
+      }
+      if (i8) {
+        // INT8 units alternate two S buffers: re-bias this warp's columns if the
+        // next user is an INT8 unit (the scores are dead now), then release
+        if (u + 2 < nu8) {
+          tmem_fill32(scol, kI8Bias);
+          tmem_fill32(scol + 32, kI8Bias);
+          tmem_wait_st();
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_P_FULL));
-        if (have_pend && !merge_x4()) { ok = false; break; }
-        have_pend = true;
-        pend_member = member;
-        pend_mb = mb;
-        pend_lb = lb;
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + (u & 1)));
       }
-      if (ok && have_pend) ok = merge_x4();
+      // the P area and the accumulator are settled once the P·V of the unit
+      // before completed
+      if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      // a rising reference first folds what the phase holds into O; INT8 also
+      // folds every 256 units, before its s32 sums could overflow
+      const bool guard = i8 && u > nu16 && ((u - nu16) & 255) == 0;
+      fold(raise || guard, i8);
+      if (raise) r_lo = r_use;
+      l_lo += lp;
+      if (present) {
+        if (i8) {
+          uint8_t* pb = smem + SM_P + half * 8192;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(pb + row * 64 + ((c ^ ((row >> 1) & 3)) * 16)) =
+                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        } else {
+          uint8_t* pb = smem + SM_P + half * 4096;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            *reinterpret_cast<uint4*>(pb + row * 32 + ((c ^ ((row >> 2) & 1)) * 16)) =
+                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+          *reinterpret_cast<uint32_t*>(smem + SM_P + PO_PSF + half * kSfAtomBytes + (row & 31) * 16 +
+                                       (row >> 5) * 4) = sfw;
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P_FULL));
+    }
+    // the last low-bit phase joins O once its last P·V completed
+    if (ok && nu > nu16) {
+      if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (nu - 1) & 1))) ok = false;
+      tc_fence_after();
+      if (ok) fold(true, nu8 == nu);
     }
     if (ok && !__all_sync(FULL, mbar_wait(bar(B_DONE), 0))) ok = false;
     tc_fence_after();
     if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
-    // ---- epilogue: O = (2^(m16-m) O + 2^(m8-m) vsc ⊙ o8) / l, vsc the channel
-    // scale of whichever low-bit phase ran last (INT8 sv or NVFP4 g)
+    // ---- epilogue: O / l in bf16, staged for the TMA store; each warp summed
+    // l over its own key blocks, against the reference both warps share
     {
-      // both halves of a row carry partial sums; exchange them
-      float* lx = red + 512;  // [2 halves][2 values][128 rows], past the item buffers
-      lx[(half * 2 + 0) * 128 + row] = l16;
-      lx[(half * 2 + 1) * 128 + row] = l8;
+      float* lx = red + 512;
+      lx[half * 128 + row] = l16;
       if (!pair_sync(B_EPI + quarter, 0)) { raise_timeout(A.status); *abort_flag = 1; }
-      const float l16t = l16 + lx[((1 - half) * 2 + 0) * 128 + row];
-      const float l8t = l8 + lx[((1 - half) * 2 + 1) * 128 + row];
-      const float mm = fmaxf(m16, m8);
-      const float a16 = m16 == -INFINITY ? 0.f : fast_exp2(m16 - mm);
-      const float a8 = m8 == -INFINITY ? 0.f : fast_exp2(m8 - mm);
-      const float lt = l16t * a16 + l8t * a8;
+      const float lt = l16 + lx[(1 - half) * 128 + row];
       const float il = lt > 0.f ? 1.0f / lt : 0.f;
       uint8_t* ot = smem + SM_Q16 + half * 16384;  // channel half = output sub-tile
 #pragma unroll
@@ -910,20 +902,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t orr[32];
         tmem_ld32(tbase + lane_off + TM_O + half * 64 + c, orr);
         tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int ch = half * 64 + c + 2 * i;
-          const float v0 = (a16 * __uint_as_float(orr[2 * i]) + a8 * vsc[ch] * o8[c + 2 * i]) * il;
-          const float v1 = (a16 * __uint_as_float(orr[2 * i + 1]) + a8 * vsc[ch + 1] * o8[c + 2 * i + 1]) * il;
-          __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
-          w[i] = *reinterpret_cast<uint32_t*>(&hb);
-        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(orr[8 * q + 2 * i]) * il,
+                                                      __uint_as_float(orr[8 * q + 2 * i + 1]) * il);
+            w[i] = *reinterpret_cast<uint32_t*>(&hb);
+          }
           const int chunk = (c >> 3) + q;
-          *reinterpret_cast<uint4*>(ot + row * 128 + ((chunk ^ (row & 7)) * 16)) =
-              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          *reinterpret_cast<uint4*>(ot + row * 128 + ((chunk ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       fence_async_smem();

@@ -7,19 +7,31 @@ quantisation scales are folded in at the phase boundaries, so no partial
 outputs are written back and merged.  Skipped pairs contribute nothing.
 
 This module follows that structure literally, per query block, in fp64:
-phase 16, then phase 8, then phase 4, key blocks in ascending index inside each
-phase, one online-softmax state (m, l, O) carried across all of them.
+phase 16, then phase 8, then phase 4, one online-softmax state (m, l, O)
+carried across all of them; each low-bit phase accumulates against its own
+power-of-two reference and is folded into that state, with its channel
+scales, at the phase boundary.
 
 Readings adopted (the pages leave these open):
 
 * scores: 16-bit phase from the bf16 values; 8-bit phase from the exact integer
   product of the INT8 codes times both block scales; 4-bit phase from the
   dequantised NVFP4 values; all times 1/sqrt(d).  Padding keys score -inf.
-* P in the 8-bit and 4-bit phases is quantised relative to the per-row maximum
-  m_blk of the key block it belongs to, p = exp(s - m_blk) in (0, 1]:
-  8-bit code = round(255 p) as an unsigned byte (scale 1/255); 4-bit = NVFP4
-  over 16 consecutive keys of the row.  The block's P·V is then weighted by
-  exp(m_blk - m) when merged into the shared accumulator.
+* key blocks are taken two at a time ("units"), in the order a kernel that
+  pairs neighbouring query blocks (2p, 2p+1) walks them: per phase, the union
+  of the two query blocks' key-block lists in ascending order, cut into
+  consecutive pairs.  A unit's blocks that this query block does not retain
+  contribute nothing to its rows.
+* P in the 8-bit and 4-bit phases is quantised relative to a running power of
+  two 2^r per row and phase (r an integer, log2 units): before a unit, if the
+  unit's row maximum x_max (of s·log2 e over its retained keys) exceeds r, r
+  becomes ceil(x_max), and what the phase accumulated so far is scaled by
+  2^(r_old - r).  So p = 2^(x - r) is in (0, 1]:
+  8-bit code = round(255 p) as an unsigned byte (scale 1/255);
+  4-bit = NVFP4, over 16 consecutive keys of the row, of 2688 p (2688 = 6·448
+  puts the largest p at the top of the e2m1 x e4m3 range), dequantised and
+  divided by 2688 again.  Each phase accumulates its P·V against its own
+  reference; the phases' results meet, with the channel scales, at the end.
 * the softmax denominator l sums the unquantised exp(s - m) over every retained
   real key of every phase.
 * 16-bit phase, ``emulate`` mode: P is rounded to bf16 relative to a power of
@@ -41,6 +53,8 @@ from . import formats as F
 from .rank import BIT4, BIT8, BIT16
 
 LOG2E = 1.4426950408889634
+LN2 = 0.6931471805599453
+P4_RANGE = 2688.0  # 6 (largest e2m1) x 448 (largest e4m3)
 
 
 def bf16_round(x):
@@ -68,6 +82,54 @@ class _State:
         self.m = m_new
 
 
+def phase_units(prec_row, partner_row, bit):
+    """The units of one phase: the key blocks that this query block or its
+    partner (the other block of its pair) assign to ``bit``, ascending, cut into
+    consecutive pairs (the last may hold one block)."""
+    sel = prec_row == bit
+    if partner_row is not None:
+        sel = sel | (partner_row == bit)
+    kbs = np.nonzero(sel)[0]
+    return [kbs[i:i + 2] for i in range(0, len(kbs), 2)]
+
+
+class _LowBitPhase:
+    """A low-bit phase's P·V accumulator and sum against a running power of two
+    2^r per row (r an integer, log2 units; -inf before the first score)."""
+
+    def __init__(self, rows, d):
+        self.r = np.full(rows, -np.inf)
+        self.l = np.zeros(rows)
+        self.acc = np.zeros((rows, d))
+
+    def enter(self, xs):
+        """Take a unit whose blocks have log2-unit scores ``xs`` ([rows, keys]
+        each, -inf where not retained): raise r to ceil of the unit's row max
+        where that max exceeds r, rescale what is accumulated, add the
+        unquantised p to l and return each block's p = 2^(x - r)."""
+        x_max = np.max(np.stack([x.max(1) for x in xs]), axis=0)
+        up = np.isfinite(x_max) & (x_max > self.r)
+        r_new = np.where(up, np.ceil(np.where(up, x_max, 0.0)), self.r)
+        had = np.isfinite(self.r)
+        a = np.where(up, np.where(had, np.exp2(np.where(had, self.r, 0.0) - np.where(up, r_new, 0.0)), 0.0), 1.0)
+        self.acc *= a[:, None]
+        self.l *= a
+        self.r = r_new
+        live = np.isfinite(self.r)
+        ps = []
+        for x in xs:
+            ok = np.isfinite(x) & live[:, None]
+            p = np.where(ok, np.exp2(np.where(ok, x - np.where(live, self.r, 0.0)[:, None], 0.0)), 0.0)
+            self.l += p.sum(1)
+            ps.append(p)
+        return ps
+
+    def fold_into(self, st, chan_scale):
+        """Phase boundary: join the shared state with the phase's channel scale."""
+        m_blk = np.where(np.isfinite(self.r), self.r * LN2, -np.inf)
+        st.merge(m_blk, self.l, self.acc * chan_scale)
+
+
 def _row_max(s):
     return s.max(axis=1)
 
@@ -78,11 +140,13 @@ def _exp_rel(s, m):
     return np.where(ok, np.exp(np.where(ok, s - np.where(np.isfinite(m), m, 0)[:, None], 0)), 0.0)
 
 
-def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
+def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None):
     """Output rows [S, d] of query block ``qb`` of one head.
 
     ``prep``: dict from ``prep.prepare_head``; ``prec_row``: uint8 [nb] precision
-    of each key block for this query block (16, 8, 4, 0)."""
+    of each key block for this query block (16, 8, 4, 0); ``partner_row``: the
+    same for the other query block of its pair (qb ^ 1), None if there is none.
+    The partner only decides how the low-bit phases group key blocks into units."""
     S = prep["q_blocks"].shape[1]
     valid = prep["valid"]
     inv_sqrt_d = 1.0 / np.sqrt(d)
@@ -113,31 +177,44 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
     # phase 8: INT8 Q/K codes with block scales, u8 P, INT8 V with channel scales
     qi = prep["q_i8"][qb].astype(np.float64)
     sq = prep["q_s8"][qb]
-    for kb in np.nonzero(prec_row == BIT8)[0]:
-        s_int = qi @ prep["k_i8"][kb].astype(np.float64).T  # exact integers
-        s = s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d)
-        s = np.where(valid[kb][None, :], s, -np.inf)
-        m_blk = _row_max(s)
-        p = _exp_rel(s, m_blk)
-        code = np.rint(255.0 * p)
-        x = (code @ prep["v_i8"][kb].astype(np.float64).T) * (prep["v_s8"][None, :] / 255.0)
-        st.merge(m_blk, p.sum(1), x)
+    ph = _LowBitPhase(S, d)
+    for unit in phase_units(prec_row, partner_row, BIT8):
+        xs = []
+        for kb in unit:
+            s_int = qi @ prep["k_i8"][kb].astype(np.float64).T  # exact integers
+            s = s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d)
+            keep = valid[kb][None, :] & (prec_row[kb] == BIT8)
+            xs.append(np.where(keep, s * LOG2E, -np.inf))
+        for kb, p in zip(unit, ph.enter(xs)):
+            code = np.rint(255.0 * p)
+            ph.acc += code @ prep["v_i8"][kb].astype(np.float64).T  # exact integers
+    ph.fold_into(st, prep["v_s8"][None, :] / 255.0)
 
-    # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks), NVFP4 V
+    # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks of 2688 p), NVFP4 V
     qd = F.nvfp4_dequantize(prep["q_f4"][qb], prep["q_sf4"][qb])
-    for kb in np.nonzero(prec_row == BIT4)[0]:
-        kd = F.nvfp4_dequantize(prep["k_f4"][kb], prep["k_sf4"][kb])
-        s = (qd @ kd.T) * inv_sqrt_d
-        s = np.where(valid[kb][None, :], s, -np.inf)
-        m_blk = _row_max(s)
-        p = _exp_rel(s, m_blk)
-        pc, psf = F.nvfp4_quantize(p, axis=-1, block=16)
-        pd = F.nvfp4_dequantize(pc, psf)
-        vt = F.nvfp4_dequantize(prep["v_f4"][kb], prep["v_sf4"][kb]) * prep["v_g4"][:, None]
-        st.merge(m_blk, p.sum(1), pd @ vt.T)
+    ph = _LowBitPhase(S, d)
+    for unit in phase_units(prec_row, partner_row, BIT4):
+        xs = []
+        for kb in unit:
+            kd = F.nvfp4_dequantize(prep["k_f4"][kb], prep["k_sf4"][kb])
+            s = (qd @ kd.T) * inv_sqrt_d
+            keep = valid[kb][None, :] & (prec_row[kb] == BIT4)
+            xs.append(np.where(keep, s * LOG2E, -np.inf))
+        for kb, p in zip(unit, ph.enter(xs)):
+            t = F.f32(P4_RANGE * F.f32(p))
+            pc, psf = F.nvfp4_quantize(t, axis=-1, block=16)
+            vt = F.nvfp4_dequantize(prep["v_f4"][kb], prep["v_sf4"][kb])
+            ph.acc += F.nvfp4_dequantize(pc, psf) @ vt.T
+    ph.fold_into(st, prep["v_g4"][None, :] / P4_RANGE)
 
     out = np.where(st.l[:, None] > 0, st.o / np.where(st.l > 0, st.l, 1.0)[:, None], 0.0)
     return bf16_round(out) if mode == "emulate" else out
+
+
+def partner_of(prec_map, qb):
+    """Precision row of the other query block of qb's pair (2p, 2p+1), or None."""
+    o = qb ^ 1
+    return prec_map[o] if o < len(prec_map) else None
 
 
 def head_attention(prep, prec_map, d, mode="emulate", qblocks=None):
@@ -145,7 +222,7 @@ def head_attention(prep, prec_map, d, mode="emulate", qblocks=None):
     nb, S = prep["valid"].shape
     out = np.zeros((nb, S, d))
     for qb in (range(nb) if qblocks is None else qblocks):
-        out[qb] = qblock_attention(prep, qb, prec_map[qb], d, mode)
+        out[qb] = qblock_attention(prep, qb, prec_map[qb], d, mode, partner_of(prec_map, qb))
     return out
 
 

@@ -77,14 +77,16 @@ def test_q_zero_closed_forms():
     vb = r["prep"]["v_i8"].astype(np.float64) * r["prep"]["v_s8"][None, :, None]  # [nb, d, S]
     vt = np.concatenate([vb[b][:, r["prep"]["valid"][b]] for b in range(p.nb)], axis=1)
     np.testing.assert_allclose(r["out"], np.broadcast_to(vt.mean(1), r["out"].shape), rtol=1e-12)
-    # 4-bit only: p = 1 → sf = e4m3(1/6) = 0.171875, code e2m1(5.818) = 6 → weight 1.03125
-    assert F.e4m3_round(1.0 / 6.0) == 0.171875
+    # 4-bit only: p = 1 is quantised as 2688 p → sf = e4m3(2688/6) = 448 (the
+    # largest e4m3), code = e2m1(2688/448) = 6 (the largest e2m1): exact, weight 1
+    assert F.e4m3_round(2688.0 / 6.0) == 448.0
+    assert F.e2m1_round(2688.0 / 448.0) == 6.0
     p4 = Problem(**{**p.__dict__, "budget": (0, 100, 0, 0)})
     r = pipeline.run_head(p4, q, k, v, mode="math")
     pr = r["prep"]
     vd = prep.dequant_v_nvfp4(pr["v_f4"], pr["v_sf4"], pr["v_g4"])
     vt = np.concatenate([vd[b][:, pr["valid"][b]] for b in range(p.nb)], axis=1)
-    np.testing.assert_allclose(r["out"], np.broadcast_to(1.03125 * vt.mean(1), r["out"].shape), rtol=1e-12)
+    np.testing.assert_allclose(r["out"], np.broadcast_to(vt.mean(1), r["out"].shape), rtol=1e-12)
 
 
 def _dequant_dense(p, pr, fmt):
@@ -147,3 +149,33 @@ def test_scatter_restores_token_order():
     x = np.random.default_rng(0).standard_normal((p.N, 4))
     blocks, _ = prep.gather_blocks(x, tab)
     np.testing.assert_array_equal(attention.scatter(blocks, tab, p.N), x)
+
+
+def test_phase_units_union_of_the_pair_in_pairs():
+    # this query block keeps 8-bit blocks 0, 2, 3; its partner 1, 3, 4
+    row = np.array([8, 0, 8, 8, 0], dtype=np.uint8)
+    partner = np.array([0, 8, 0, 8, 8], dtype=np.uint8)
+    units = [list(u) for u in attention.phase_units(row, partner, 8)]
+    assert units == [[0, 1], [2, 3], [4]]
+    assert [list(u) for u in attention.phase_units(row, None, 8)] == [[0, 2], [3]]
+
+
+def test_low_bit_reference_raise_by_hand():
+    # one row; unit 1 max 0.3 → r = ceil(0.3) = 1; unit 2 max 2.5 → r = 3 and
+    # what unit 1 left is scaled by 2^(1-3)
+    ph = attention._LowBitPhase(1, 2)
+    (p1,) = ph.enter([np.array([[0.3, -np.inf]])])
+    assert ph.r[0] == 1.0
+    assert p1[0, 0] == 2.0 ** (0.3 - 1.0) and p1[0, 1] == 0.0
+    c1 = np.rint(255.0 * p1)  # 157
+    assert c1[0, 0] == 157.0
+    ph.acc += c1[:, :1] * np.array([[10.0, -20.0]])
+    (pa, pb) = ph.enter([np.array([[2.5]]), np.array([[-1.0]])])
+    assert ph.r[0] == 3.0
+    np.testing.assert_allclose(ph.acc, [[157.0 * 10.0 / 4.0, -157.0 * 20.0 / 4.0]], rtol=0, atol=0)
+    assert pa[0, 0] == 2.0 ** -0.5 and pb[0, 0] == 2.0 ** -4.0
+    np.testing.assert_allclose(ph.l, [2.0 ** (0.3 - 1.0) / 4.0 + 2.0 ** -0.5 + 2.0 ** -4.0], rtol=1e-15)
+    # a unit below the reference leaves it alone; an all -inf unit changes nothing
+    ph.enter([np.array([[1.0]])])
+    ph.enter([np.array([[-np.inf]])])
+    assert ph.r[0] == 3.0
