@@ -531,8 +531,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_st32(tbase + lane_off + TM_O + half * 64 + 32, z);
       tmem_wait_st();
     }
+    // item entries (and INT8 key scales) are loaded one unit ahead, so no unit
+    // starts by waiting on global memory
+    auto item_for = [&](int v) -> uint32_t {
+      if (v >= nu) return 0u;
+      int i0v, cntv;
+      unit_items(v, i0v, cntv);
+      return half < cntv ? items[i0v + half] : 0u;
+    };
+    auto sk_for = [&](int v, uint32_t ev) -> float {
+      return (v >= nu16 && v < nu8) ? A.k_s8[(size_t)bh * g.nb + item_kb(ev)] : 0.f;
+    };
+    uint32_t e_next = item_for(0);
+    float sk_next = sk_for(0, e_next);
     for (int u = 0; ok && u < nu16; ++u) {
-      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
       const int b = u & 1;
       int i0, cnt;
       unit_items(u, i0, cnt);
@@ -542,7 +555,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_after();
         // ---- 16-bit unit: this warp owns key block `half` of the unit
         const bool present = half < cnt;
-        const uint32_t e = present ? items[i0 + half] : 0u;
+        const uint32_t e = e_next;
+        e_next = item_for(u + 1);
         const bool member = present && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
         uint32_t sr[64];
         if (present) {
@@ -575,6 +589,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         xch[half * 128 + row] = mx;
         if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+        sk_next = sk_for(u + 1, e_next);  // the entry has arrived by now; the scale has a unit's time
         mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * sl2;  // unit row max, log2 units
         const bool row_live = mx != -INFINITY;  // the row is a member of some block of the unit
         const bool need = row_live && (mx > m16 + kRescaleThreshold || m16 == -INFINITY);
@@ -677,7 +692,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_st();
     };
     for (int u = nu16; ok && u < nu; ++u) {
-      if (__any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
+      if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
       const bool i8 = u < nu8;
       if (u == nu8 && nu8 > nu16) {
         // INT8 -> 4-bit boundary: the INT8 accumulator joins O once its last
@@ -691,10 +706,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       unit_items(u, i0, cnt);
       // ---- this warp's block of the unit: key block `half`, all 64 keys
       const bool present = half < cnt;
-      const uint32_t e = present ? items[i0 + half] : 0u;
+      const uint32_t e = e_next;
+      const float sk = sk_next;
+      e_next = item_for(u + 1);
       const int kb = item_kb(e);
       const bool member = present && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
-      const float sk = (i8 && present) ? A.k_s8[(size_t)bh * g.nb + kb] : 0.f;  // issued before the wait
       if (u == nu8 && half == 0) {
         // first 4-bit unit: Q's scale factors into TMEM (each lane quarter
         // holds all 128 rows).  The columns were the second S buffer, whose
@@ -765,6 +781,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       xch[half * 128 + row] = mx;
       if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+      sk_next = sk_for(u + 1, e_next);  // the entry has arrived by now; the scale has a unit's time
       mx = fmaxf(mx, xch[(1 - half) * 128 + row]);  // the unit's row maximum
       // the reference rises to ceil(max) whenever the max exceeds it
       const bool raise = mx != -INFINITY && (r_lo == -INFINITY || mx > r_lo);
@@ -1041,6 +1058,19 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t rowbytes
 }
 
 }  // namespace
+
+bool tma_available() { return encode_fn() != nullptr; }
+
+bool make_region_map(CUtensorMap* m, const void* base, const Geom& g, bool swizzle128) {
+  const cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.Ww, (cuuint64_t)g.Hh, (cuuint64_t)g.BH * g.T};
+  const cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.Ww * g.d * 2, (cuuint64_t)g.Hh * g.Ww * g.d * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)g.rw, (cuuint32_t)g.rh, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return encode_fn() && encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool attention_tc_supported(const Geom& g) {
   return g.d == kD && encode_fn() != nullptr;

@@ -2,6 +2,7 @@
 // geometry, workspace layout and small device helpers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -184,6 +185,11 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k,
                          const void* v, void* out, cudaStream_t st);
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st);
+// TMA: whether the driver's tensor-map encoder was found, and the 4-D view
+// [B*H*T][Hh][Ww][d] of a bf16 [B,H,N,d] tensor in {64 channels, rw, rh, 1}
+// region boxes (zero fill outside the frame).
+bool tma_available();
+bool make_region_map(CUtensorMap* m, const void* base, const Geom& g, bool swizzle128);
 bool attention_tc_supported(const Geom& g);
 cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, const void* k,
                                 const void* v, void* ws, void* out, cudaStream_t st);
