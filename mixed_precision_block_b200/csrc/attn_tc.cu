@@ -55,6 +55,7 @@
 #include <cuda.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "da2_internal.cuh"
 #include "sm100.cuh"
@@ -214,6 +215,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto bar = [&](int i) { return s0 + SM_BAR + 8u * (uint32_t)i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 8);
+  // 1 / (1 + m/8) for m = 0..7, then 1 / m (0 for m = 0): reciprocals of e4m3 scales
+  float* rcp_tab = reinterpret_cast<float*>(smem + SM_MISC + 64);
+  if (threadIdx.x < 16)
+    rcp_tab[threadIdx.x] = threadIdx.x < 8 ? 8.0f / (float)(8 + threadIdx.x)
+                                           : (threadIdx.x > 8 ? 1.0f / (float)(threadIdx.x - 8) : 0.f);
 
   // units: each phase takes its items (key blocks) two at a time, in list order
   const int nu16 = (n16 + 1) / 2;
@@ -691,13 +697,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       tmem_wait_st();
     };
-    for (int u = nu16; ok && u < nu; ++u) {
-      if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-      const bool i8 = u < nu8;
-      if (u == nu8 && nu8 > nu16) {
+    // one low-bit unit, instantiated once per format so that each phase's
+    // loop holds only its own code
+    auto lowbit_unit = [&](const int u, auto fmt) -> bool {
+      constexpr bool i8 = decltype(fmt)::value;
+      if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) return false;
+      if (!i8 && u == nu8 && nu8 > nu16) {
         // INT8 -> 4-bit boundary: the INT8 accumulator joins O once its last
         // P·V completed; the columns then start the 4-bit accumulator at zero
-        if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+        if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (u - 1) & 1))) return false;
         tc_fence_after();
         fold(true, true);
         r_lo = -INFINITY;
@@ -711,7 +719,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       e_next = item_for(u + 1);
       const int kb = item_kb(e);
       const bool member = present && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
-      if (u == nu8 && half == 0) {
+      if (!i8 && u == nu8 && half == 0) {
         // first 4-bit unit: Q's scale factors into TMEM (each lane quarter
         // holds all 128 rows).  The columns were the second S buffer, whose
         // scores this warp has read, and no S MMA writes there any more.
@@ -736,7 +744,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(bar(B_SFQ));
       }
       float* xch = red + (u & 1) * 256;  // [2 halves][128 rows] for this unit
-      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1))) { ok = false; break; }
+      if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1))) return false;
       tc_fence_after();
       // this warp's scores: 64 columns of the unit's S buffer
       const uint32_t scol = tbase + lane_off + TM_S + (i8 ? (uint32_t)(u & 1) * 128u : 0u) + half * 64;
@@ -780,7 +788,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (lane == 0) mbar_arrive(bar(B_S_FREE + (u & 1)));
       }
       xch[half * 128 + row] = mx;
-      if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) { ok = false; break; }
+      if (!pair_sync(B_PAIR + quarter * 2 + (u & 1), (u >> 1) & 1)) return false;
       sk_next = sk_for(u + 1, e_next);  // the entry has arrived by now; the scale has a unit's time
       mx = fmaxf(mx, xch[(1 - half) * 128 + row]);  // the unit's row maximum
       // the reference rises to ceil(max) whenever the max exceeds it
@@ -837,8 +845,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               pm = fmax3(pm, __uint_as_float(sr[16 * mbk + i]), __uint_as_float(sr[16 * mbk + i + 1]));
             const uint32_t sf = cvt_e4m3x2(0.0f, (pm * kP4Range) * (1.0f / 6.0f)) & 0xffu;
             sfw |= sf << (8 * mbk);
-            const float dec = e4m3_to_f32(sf);
-            const float rr = dec != 0.f ? kP4Range * __frcp_rn(dec) : 0.f;
+            // 2688 / sf without the SFU: sf = 2^(e-7) (1 + m/8), or m 2^-9 when e = 0
+            const uint32_t ex = sf >> 3, mt = sf & 7u;
+            const float inv_m = rcp_tab[ex ? mt : 8u + mt];
+            const float rr = kP4Range * inv_m * __uint_as_float((ex ? 134u - ex : 136u) << 23);
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
               uint32_t w = 0;
@@ -866,7 +876,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // the P area and the accumulator are settled once the P·V of the unit
       // before completed
-      if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
+      if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) return false;
       tc_fence_after();
       // a rising reference first folds what the phase holds into O; INT8 also
       // folds every 256 units, before its s32 sums could overflow
@@ -895,7 +905,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_P_FULL));
-    }
+      return true;
+    };
+    for (int u = nu16; ok && u < nu8; ++u) ok = lowbit_unit(u, std::true_type{});
+    for (int u = nu8; ok && u < nu; ++u) ok = lowbit_unit(u, std::false_type{});
     // the last low-bit phase joins O once its last P·V completed
     if (ok && nu > nu16) {
       if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (nu - 1) & 1))) ok = false;
