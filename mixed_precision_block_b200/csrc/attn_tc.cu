@@ -121,7 +121,7 @@ constexpr uint32_t TM_SFQ = 256, TM_SFK = 264, TM_SFV = 280, TM_SFP = 288;
 enum {
   B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
   B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages,
-  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 1, B_DONE = B_P_FREE + 1,
+  B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_P_FREE = B_P_FULL + 2, B_DONE = B_P_FREE + 2,
   B_PAIR = B_DONE + 1,   // [4 quarters][2 parities]: the two warps of a row quarter
   B_EPI = B_PAIR + 8,    // [4 quarters]: final exchange
   B_COUNT = B_EPI + 4
@@ -230,6 +230,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     else if (u < nu8) { i0 = n16 + 2 * (u - nu16); cnt = min(2, n16 + n8 - i0); }
     else { i0 = n16 + n8 + 2 * (u - nu8); cnt = min(2, n16 + n8 + n4 - i0); }
   };
+  // an INT8 unit's S buffer holds the bias (1.5*2^23 as s32) unless a 16-bit
+  // unit's P was the last thing in it
+  auto i8_biased = [&](int u) { return u < 2 || u - 2 >= nu16; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q16), 1);
@@ -244,8 +247,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(B_S_FULL + b), 1);
       mbar_init(bar(B_S_FREE + b), kSoftmaxWarps);
     }
-    mbar_init(bar(B_P_FULL), kSoftmaxWarps);
-    mbar_init(bar(B_P_FREE), 1);
+    for (int b = 0; b < 2; ++b) {  // per unit parity: P of unit u, P·V of unit u
+      mbar_init(bar(B_P_FULL + b), kSoftmaxWarps);
+      mbar_init(bar(B_P_FREE + b), 1);
+    }
     mbar_init(bar(B_DONE), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(B_PAIR + i), 2);
     for (int i = 0; i < 4; ++i) mbar_init(bar(B_EPI + i), 2);
@@ -415,8 +420,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // 16-bit and INT8 units alternate two S buffers; 4-bit units share
           // one (the second holds scale factors), so they wait for the unit
           // before — for the first of them that implies both buffers were read
-          const bool s_free = single ? (sn < 1 || mbar_test(bar(B_S_FREE + ((sn - 1) & 1)), ((sn - 1) >> 1) & 1))
-                                     : (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1));
+          // A 16-bit unit's P lives in its S buffer until its P·V completes.
+          auto pv_done = [&](int j) {
+            return j < 0 || j >= nu16 || mbar_test(bar(B_P_FREE + (j & 1)), (j >> 1) & 1);
+          };
+          const bool s_free = single ? (sn < 1 || mbar_test(bar(B_S_FREE + ((sn - 1) & 1)), ((sn - 1) >> 1) & 1)) &&
+                                           pv_done(sn - 1) && pv_done(sn - 2)
+                                     : (sn < 2 || mbar_test(bar(B_S_FREE + b), ((sn >> 1) - 1) & 1)) && pv_done(sn - 2);
           if ((sn < nu8 || f4_ready) && s_free && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1)) {
             tc_fence_after();
             const uint32_t st = s0 + SM_K + s * 32768;
@@ -436,7 +446,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
-                       smem_desc(st + kk * 32, 16, 1024, SW_128), id, 1u);  // onto the bias
+                       smem_desc(st + kk * 32, 16, 1024, SW_128), id,
+                       (kk > 0 || i8_biased(sn)) ? 1u : 0u);  // onto the bias where it was laid
             } else {
               for (int t = 0; t < cnt; ++t) {
                 const uint32_t sfk = tbase + TM_SFK + 8 * t;
@@ -459,18 +470,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int s = pn % kStages;
           const bool low = pn >= nu16;  // INT8 or 4-bit: P·V accumulates at TM_ACC
           // (the softmax warps settle the accumulator before they release P)
-          if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL), pn & 1)) {
+          if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) &&
+              mbar_test(bar(B_P_FULL + (pn & 1)), (pn >> 1) & 1)) {
             tc_fence_after();
             const uint32_t st = s0 + SM_V + s * 32768;
             const uint32_t pbuf = s0 + SM_P;
             if (!low) {
               int i0, cnt;
               unit_items(pn, i0, cnt);
+              // P of block t sits in TMEM, in block t's own score columns
+              const uint32_t pt = tbase + TM_S + (pn & 1) * 128;
               for (int t = 0; t < cnt; ++t) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                  mma_f16(tbase + TM_O, smem_desc(pbuf + t * 16384 + kk * 32, 16, 1024, SW_128),
-                          smem_desc(st + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
+                  mma_f16_ta(tbase + TM_O, pt + 64 * t + 8 * kk,
+                             smem_desc(st + t * 16384 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
               }
             } else if (pn < nu8) {
               int i0, cnt;
@@ -492,7 +506,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                        smem_desc(st + t * 4096, 16, 256, SW_32), id4pv, 1u, sfp, sfv);
               }
             }
-            mma_commit(bar(B_P_FREE));
+            mma_commit(bar(B_P_FREE + (pn & 1)));
             mma_commit(bar(B_V_EMPTY + s));
             ++pn;
             progressed = true;
@@ -526,6 +540,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(idx));
       return __all_sync(FULL, mbar_wait(bar(idx), parity));
+    };
+    // the P·V of unit v (and every MMA before it) has completed
+    auto pfree_wait = [&](int v) -> bool {
+      return v < 0 || mbar_wait(bar(B_P_FREE + (v & 1)), (uint32_t)(v >> 1) & 1u);
     };
     float m16 = -INFINITY, l16 = 0.f;  // 16-bit phase: O in TMEM, integer reference
     bool ok = true;
@@ -569,11 +587,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tmem_ld32(sbase + half * 64, sr);
           tmem_ld32(sbase + half * 64 + 32, sr + 32);
           tmem_wait_ld();
-        }
-        if (u + 2 >= nu16 && u + 2 < nu8) {  // the buffer's next user is an INT8 unit
-          tmem_fill32(sbase + half * 64, kI8Bias);
-          tmem_fill32(sbase + half * 64 + 32, kI8Bias);
-          tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
@@ -626,10 +639,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int i = 0; i < 32; ++i) pw[i] = 0u;
           l16 *= a;
         }
-        // the P buffer and O are free once the P·V of unit u-1 completed
-        if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) { ok = false; break; }
-        tc_fence_after();
+        // O can be rescaled once the P·V of unit u-1 completed; only then wait
         if (__any_sync(FULL, need_o)) {
+          if (!__all_sync(FULL, pfree_wait(u - 1))) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 64; c += 32) {
             uint32_t orr[32];
@@ -641,17 +654,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           tmem_wait_st();
         }
+        // P (bf16 pairs, key 2i in the low half of column i) replaces this
+        // warp's own scores in TMEM, where the P·V MMA reads it
         if (present) {
-          uint8_t* pb = smem + SM_P + half * 16384;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(pb + row * 128 + ((c ^ (row & 7)) * 16)) =
-                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+          tmem_st32(sbase + half * 64, pw);
+          tmem_wait_st();
         }
-      fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL));
+      if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
     }
     // ================================================================ low-bit phases
     // Each low-bit phase accumulates P·V in TMEM (INT8: s32 X8; 4-bit: fp32
@@ -705,7 +716,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!i8 && u == nu8 && nu8 > nu16) {
         // INT8 -> 4-bit boundary: the INT8 accumulator joins O once its last
         // P·V completed; the columns then start the 4-bit accumulator at zero
-        if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (u - 1) & 1))) return false;
+        if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
         tc_fence_after();
         fold(true, true);
         r_lo = -INFINITY;
@@ -759,8 +770,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_ld32(scol + 32, sr + 32);
         tmem_wait_ld();
         if (i8) {
-          // the s32 scores sit on the bias: subtracting it gives them exactly (|S| < 128*127^2 < 2^22)
+          // the s32 scores sit on the bias (or are put on it, where a 16-bit
+          // unit used the buffer last): subtracting it gives them exactly
+          // (|S| < 128*127^2 < 2^22)
           const uint64_t kx2 = f2pack(-kI8BiasF, -kI8BiasF);
+          if (!i8_biased(u)) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) sr[i] += kI8Bias;
+          }
 #pragma unroll
           for (int i = 0; i < 64; i += 2) {
             float a, b;
@@ -876,7 +893,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // the P area and the accumulator are settled once the P·V of the unit
       // before completed
-      if (!__all_sync(FULL, u < 1 || mbar_wait(bar(B_P_FREE), (u - 1) & 1))) return false;
+      if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
       tc_fence_after();
       // a rising reference first folds what the phase holds into O; INT8 also
       // folds every 256 units, before its s32 sums could overflow
@@ -904,14 +921,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL));
+      if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
       return true;
     };
     for (int u = nu16; ok && u < nu8; ++u) ok = lowbit_unit(u, std::true_type{});
     for (int u = nu8; ok && u < nu; ++u) ok = lowbit_unit(u, std::false_type{});
     // the last low-bit phase joins O once its last P·V completed
     if (ok && nu > nu16) {
-      if (!__all_sync(FULL, mbar_wait(bar(B_P_FREE), (nu - 1) & 1))) ok = false;
+      if (!__all_sync(FULL, pfree_wait(nu - 1))) ok = false;
       tc_fence_after();
       if (ok) fold(true, nu8 == nu);
     }

@@ -185,6 +185,14 @@ __device__ __forceinline__ void mma_f16(uint32_t dtmem, uint64_t adesc, uint64_t
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(id), "r"(acc));
 }
+// kind::f16 with the A operand (M rows x K, 16-bit, two per 32-bit column)
+// read from tensor memory instead of shared memory.
+__device__ __forceinline__ void mma_f16_ta(uint32_t dtmem, uint32_t atmem, uint64_t bdesc, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(dtmem), "r"(atmem), "l"(bdesc), "r"(id), "r"(acc));
+}
 __device__ __forceinline__ void mma_i8(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t id, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
