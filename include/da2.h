@@ -109,10 +109,14 @@ int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
 /* Stage 3 ([abstract]; [note] Method overview bullet 4; [v1] order restore).
  * Per query block one pass runs the 16-bit phase (bf16 Q/K/V), the INT8 phase
  * and the NVFP4 phase over its assigned key blocks with one shared online
- * softmax state and one fp32 accumulator; low-bit P is quantised relative to
- * each key block's row maximum; quantisation scales are applied when a block
- * is merged.  The output rows are written straight back to the original token
- * order (padding rows dropped); a query block with no key block outputs zeros.
+ * softmax state and one fp32 output accumulator.  Key blocks are taken two at
+ * a time over the merged lists of the query-block pair (2p, 2p+1); low-bit P
+ * is quantised against a running power of two per row and phase, raised per
+ * such unit to the ceiling of the unit's row maximum (4-bit P as NVFP4 of
+ * 2688 p), and each low-bit phase joins the shared accumulator with its
+ * channel scale at the phase boundary.  The output rows are written straight
+ * back to the original token order (padding rows dropped); a query block with
+ * no key block outputs zeros.
  * q, k, v: the same device tensors given to da2_prepare; out: device bf16
  * [B,H,N,d].  Requires da2_draft_rank (or da2_rank_from_scores) first. */
 int da2_attention(const da2_problem* p, const void* q, const void* k, const void* v,
@@ -120,7 +124,10 @@ int da2_attention(const da2_problem* p, const void* q, const void* k, const void
 
 /* Own dense bf16 softmax attention over all N tokens (the comparison point
  * for the sparse path): out = softmax(q k^T / sqrt d) v, fp32 accumulation,
- * bf16 output.  q, k, v, out: device bf16 [B,H,N,d]; d in {64,128}. */
+ * bf16 output.  q, k, v, out: device bf16 [B,H,N,d]; d in {64,128}.  For
+ * d = 128 (N >= 64, B*H <= 65535) it runs the sparse path's tensor-core
+ * kernel with every key block in the 16-bit phase, over 64-token blocks in
+ * natural order; otherwise a warp-MMA kernel.  Needs no workspace. */
 int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k,
                         const void* v, void* out, void* stream);
 

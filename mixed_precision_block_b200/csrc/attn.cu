@@ -650,6 +650,7 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
 
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k, const void* v, void* out,
                          cudaStream_t st) {
+  if (dense_tc_supported(B, H, N, d)) return launch_dense_tc(B, H, N, q, k, v, out, st);
   return d == 128 ? launch_dense_d<128>(B, H, N, q, k, v, out, st)
                   : launch_dense_d<64>(B, H, N, q, k, v, out, st);
 }

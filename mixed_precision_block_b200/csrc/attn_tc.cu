@@ -140,6 +140,7 @@ struct TcArgs {
   const uint8_t* v_sf4;
   int* status;
   int npairs;
+  int dense;  // every key block in the 16-bit phase; no item lists are read
 };
 
 __device__ __forceinline__ void raise_timeout(int* status) { atomicOr(status, 1); }
@@ -209,9 +210,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qa = 2 * pair, qb = (2 * pair + 1 < g.nb) ? 2 * pair + 1 : -1;
   const size_t prow = (size_t)bh * A.npairs + pair;
-  const int4 pc = *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
+  const int4 pc = A.dense ? make_int4(g.nb, 0, 0, 0) : *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
   const int n16 = pc.x, n8 = pc.y, n4 = pc.z;
-  const uint32_t* items = A.plist + prow * (size_t)(2 * g.nb);
+  const uint32_t* items = A.dense ? nullptr : A.plist + prow * (size_t)(2 * g.nb);
+  // entry i of the pair's list; in dense mode key block i, kept by both query
+  // blocks, flagged full unless it holds the ragged tail
+  auto item_at = [&](int i) -> uint32_t {
+    if (!A.dense) return items[i];
+    return (uint32_t)i | (1u << 16) | ((2 * pair + 1 < g.nb ? 1u : 0u) << 17) |
+           ((uint32_t)((i + 1) * 64 <= g.N) << 20);
+  };
   auto bar = [&](int i) { return s0 + SM_BAR + 8u * (uint32_t)i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 8);
@@ -258,7 +266,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(s0 + SM_MISC, 512);
-  if (threadIdx.x < kD) {
+  if (threadIdx.x < kD && !A.dense) {
     const float sv = A.v_s8[(size_t)bh * kD + threadIdx.x], gv = A.v_g4[(size_t)bh * kD + threadIdx.x];
     float* vsc = reinterpret_cast<float*>(smem + SM_VS);
     vsc[VS_SV255 / 4 + threadIdx.x] = sv / 255.0f;
@@ -336,18 +344,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (kn < nu16) {
             mbar_expect_tx(fb, 16384u * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t) {
-              box(item_kb(items[i0 + t]), cx, cy, cf);
+              box(item_kb(item_at(i0 + t)), cx, cy, cf);
               tma_load_4d(dst + t * 8192, &tmK, fb, 0, cx, cy, cf);
               tma_load_4d(dst + 16384 + t * 8192, &tmK, fb, 64, cx, cy, cf);
             }
           } else if (kn < nu8) {
             mbar_expect_tx(fb, 8192u * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t)
-              tma_load_2d(dst + t * 8192, &tmK8, fb, 0, (bh * g.nb + item_kb(items[i0 + t])) * 64);
+              tma_load_2d(dst + t * 8192, &tmK8, fb, 0, (bh * g.nb + item_kb(item_at(i0 + t))) * 64);
           } else {
             mbar_expect_tx(fb, (4096u + 2 * kSfAtomBytes) * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t) {
-              const size_t kl = (size_t)bh * g.nb + item_kb(items[i0 + t]);
+              const size_t kl = (size_t)bh * g.nb + item_kb(item_at(i0 + t));
               tma_load_2d(dst + t * 4096, &tmK4, fb, 0, (int)(kl * 64));
               bulk_load(dst + SL_SF + t * 2 * kSfAtomBytes, A.k_sf4 + kl * 2 * kSfAtomBytes, 2 * kSfAtomBytes, fb);
             }
@@ -363,18 +371,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (vn < nu16) {
             mbar_expect_tx(fb, 16384u * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t) {
-              box(item_kb(items[i0 + t]), cx, cy, cf);
+              box(item_kb(item_at(i0 + t)), cx, cy, cf);
               tma_load_4d(dst + t * 16384, &tmV, fb, 0, cx, cy, cf);
               tma_load_4d(dst + t * 16384 + 8192, &tmV, fb, 64, cx, cy, cf);
             }
           } else if (vn < nu8) {
             mbar_expect_tx(fb, 8192u * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t)
-              tma_load_2d(dst + t * 8192, &tmV8, fb, 0, (bh * g.nb + item_kb(items[i0 + t])) * kD);
+              tma_load_2d(dst + t * 8192, &tmV8, fb, 0, (bh * g.nb + item_kb(item_at(i0 + t))) * kD);
           } else {
             mbar_expect_tx(fb, (4096u + kSfAtomBytes) * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t) {
-              const size_t kl = (size_t)bh * g.nb + item_kb(items[i0 + t]);
+              const size_t kl = (size_t)bh * g.nb + item_kb(item_at(i0 + t));
               tma_load_2d(dst + t * 4096, &tmV4, fb, 0, (int)(kl * kD));
               bulk_load(dst + SL_SF + t * kSfAtomBytes, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
             }
@@ -561,7 +569,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (v >= nu) return 0u;
       int i0v, cntv;
       unit_items(v, i0v, cntv);
-      return half < cntv ? items[i0v + half] : 0u;
+      return half < cntv ? item_at(i0v + half) : 0u;
     };
     auto sk_for = [&](int v, uint32_t ev) -> float {
       return (v >= nu16 && v < nu8) ? A.k_s8[(size_t)bh * g.nb + item_kb(ev)] : 0.f;
@@ -1103,7 +1111,41 @@ bool make_region_map(CUtensorMap* m, const void* base, const Geom& g, bool swizz
 }
 
 bool attention_tc_supported(const Geom& g) {
-  return g.d == kD && encode_fn() != nullptr;
+  return g.d == kD && g.BH <= 65535 && encode_fn() != nullptr;
+}
+
+// Status word of the dense path (its waits are bounded like the sparse path's;
+// the dense entry point has no workspace to report through).
+__device__ int g_dense_status;
+
+bool dense_tc_supported(int B, int H, int N, int d) {
+  return d == kD && N >= 64 && (long long)B * H <= 65535 && encode_fn() != nullptr;
+}
+
+// Dense attention on the same kernel: the token axis viewed as one frame of
+// 1 x N tokens cut into 64-token regions (natural order), every key block in
+// the 16-bit phase, the tail block masked and clipped by TMA like a padded region.
+cudaError_t launch_dense_tc(int B, int H, int N, const void* q, const void* k, const void* v, void* out,
+                            cudaStream_t st) {
+  Geom g{};
+  g.B = B; g.H = H; g.T = 1; g.Hh = 1; g.Ww = N; g.d = kD; g.rh = 1; g.rw = 64;
+  g.nry = 1; g.nrx = (N + 63) / 64; g.nb = g.nrx; g.N = N; g.BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (!map_regions(&tq, q, g) || !map_regions(&tk, k, g) || !map_regions(&tv, v, g) || !map_regions(&to, out, g))
+    return cudaErrorInvalidValue;
+  int* status = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_dense_status);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(status, 0, sizeof(int), st)) != cudaSuccess) return e;
+  TcArgs A{};
+  A.status = status;
+  A.npairs = (g.nb + 1) / 2;
+  A.dense = 1;
+  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // the low-bit tensor maps are never used in dense mode
+  attn_tc_kernel<<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq, tk, tv, tq, tk, tv, g, A);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st) {

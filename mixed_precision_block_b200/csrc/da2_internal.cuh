@@ -189,6 +189,9 @@ cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStre
 // [B*H*T][Hh][Ww][d] of a bf16 [B,H,N,d] tensor in {64 channels, rw, rh, 1}
 // region boxes (zero fill outside the frame).
 bool tma_available();
+bool dense_tc_supported(int B, int H, int N, int d);
+cudaError_t launch_dense_tc(int B, int H, int N, const void* q, const void* k, const void* v, void* out,
+                            cudaStream_t st);
 bool make_region_map(CUtensorMap* m, const void* base, const Geom& g, bool swizzle128);
 bool attention_tc_supported(const Geom& g);
 cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, const void* k,

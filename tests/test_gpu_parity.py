@@ -107,7 +107,7 @@ def test_full_dense_budget_matches_own_dense_kernel():
     assert PT.rel_l2(a, b) < 1e-3
 
 
-@pytest.mark.parametrize("N,d", [(1000, 128), (64, 64), (4097, 128), (130, 64)])
+@pytest.mark.parametrize("N,d", [(1000, 128), (64, 64), (4097, 128), (130, 64), (64, 128), (191, 128)])
 def test_dense_kernel_against_fp64(N, d):
     g = torch.Generator(device="cuda").manual_seed(N + d)
     q, k, v = (torch.randn((1, 2, N, d), generator=g, device="cuda") * s for s in (1.0, 1.0, 1.0))
