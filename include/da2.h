@@ -48,7 +48,8 @@ enum {
   DA2_ERR_ARG = 1,          /* invalid sizes, pointers, lambda or budget       */
   DA2_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, rh*rw != 64, no sm_100 GPU    */
   DA2_ERR_WORKSPACE = 3,    /* workspace NULL, misaligned or too small         */
-  DA2_ERR_CUDA = 4          /* a CUDA launch or runtime call failed            */
+  DA2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed            */
+  DA2_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (see below)  */
 };
 
 /* Problem statement of one attention call.
@@ -193,6 +194,13 @@ int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, ui
                      int32_t* counts, void* stream);
 
 /* Human-readable name of a status code (static string). */
+/* Device status of the last da2_attention on `ws`: synchronises `stream`, reads
+ * the workspace status word and returns DA2_OK, or DA2_ERR_TIMEOUT if a
+ * bounded wait inside the attention kernel expired (the call's output is then
+ * incomplete), or DA2_ERR_CUDA if the stream reports an error.  No counterpart
+ * on the pages: it reports this implementation's own wait bounds. */
+int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void* stream);
+
 const char* da2_status_string(int status);
 
 #ifdef __cplusplus

@@ -180,6 +180,20 @@ int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, ui
   return cuda_status(launch_rank_noalloc(g, scores, map, lists, counts, (cudaStream_t)stream));
 }
 
+int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  const Layout L = make_layout(g);
+  if (!ws || ws_bytes < L.total) return DA2_ERR_WORKSPACE;
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, static_cast<const char*>(ws) + L.off[R_STATUS], sizeof(int),
+                                  cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  return word ? DA2_ERR_TIMEOUT : DA2_OK;
+}
+
 const char* da2_status_string(int s) {
   switch (s) {
     case DA2_OK: return "ok";
@@ -187,6 +201,7 @@ const char* da2_status_string(int s) {
     case DA2_ERR_UNSUPPORTED: return "unsupported problem or device";
     case DA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case DA2_ERR_CUDA: return "CUDA launch or runtime error";
+    case DA2_ERR_TIMEOUT: return "a bounded wait in the attention kernel expired";
     default: return "unknown status";
   }
 }

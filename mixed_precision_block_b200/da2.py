@@ -20,13 +20,14 @@ if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m mixed_precision_block_b200.build`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
-DA2_OK, DA2_ERR_ARG, DA2_ERR_UNSUPPORTED, DA2_ERR_WORKSPACE, DA2_ERR_CUDA = range(5)
+DA2_OK, DA2_ERR_ARG, DA2_ERR_UNSUPPORTED, DA2_ERR_WORKSPACE, DA2_ERR_CUDA, DA2_ERR_TIMEOUT = range(6)
 
 VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_S8",
          "Q_F4", "K_F4", "Q_SF4", "K_SF4", "V_I8", "V_S8", "V_F4", "V_SF4", "V_G4",
          "SCORES", "MAP", "LISTS", "COUNTS", "STATUS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
-           "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_status_string"]
+           "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_check_status",
+           "da2_status_string"]
 NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
 
 
@@ -65,6 +66,7 @@ _lib.da2_attention.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.da2_dense_attention.argtypes = [ctypes.c_int] * 4 + [_vp] * 5
 _lib.da2_debug_view.argtypes = [_P, _vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]
 _lib.da2_rank_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
+_lib.da2_check_status.argtypes = [_P, _vp, _sz, _vp]
 _lib.da2_status_string.argtypes = [ctypes.c_int]
 _lib.da2_status_string.restype = ctypes.c_char_p
 for _f in EXPORTS[:-1]:
@@ -135,6 +137,12 @@ def da2_rank_noalloc(p, scores, prec_map, lists, counts, stream=None):
 def da2_attention(p, q, k, v, ws, out, stream=None):
     _check("da2_attention", _lib.da2_attention(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(ws),
                                                ws.numel(), _ptr(out), _stream(stream, ws)))
+
+
+def da2_check_status(p, ws, stream=None):
+    """Synchronise `stream` and return the status of the last attention on `ws`
+    (0, or DA2_ERR_TIMEOUT = 5 if a bounded wait in the kernel expired)."""
+    return _lib.da2_check_status(ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream, ws))
 
 
 def da2_dense_attention(q, k, v, out, stream=None):

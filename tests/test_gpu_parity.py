@@ -48,6 +48,7 @@ def _full_check(wl, heads=None, dense_ref=True):
             dn = PT.dense_rows(qh, kh, vh, toks)
             outs.append(PT.rel_l2(got, dn))
     assert int(da2.view(p, ws, "STATUS")[0]) == 0
+    assert da2.da2_check_status(p, ws) == 0
     return outs
 
 

@@ -86,6 +86,8 @@ def test_entry_points_check_workspace_and_pointers_before_launch(da2):
     assert lib.da2_attention(ctypes.byref(p), fake, fake, fake, fake, big, None, None) == da2.DA2_ERR_ARG
     assert lib.da2_dense_attention(1, 1, 64, 96, fake, fake, fake, fake, None) == da2.DA2_ERR_UNSUPPORTED
     assert lib.da2_dense_attention(1, 1, 0, 64, fake, fake, fake, fake, None) == da2.DA2_ERR_ARG
+    assert lib.da2_check_status(ctypes.byref(p), None, big, None) == da2.DA2_ERR_WORKSPACE
+    assert lib.da2_check_status(ctypes.byref(p), fake, big - 1, None) == da2.DA2_ERR_WORKSPACE
 
 
 def test_workspace_views_are_disjoint_and_inside(da2):
@@ -108,3 +110,4 @@ def test_status_strings(da2):
     assert da2.da2_status_string(0) == "ok"
     assert "workspace" in da2.da2_status_string(3)
     assert da2.da2_status_string(99) == "unknown status"
+    assert "bounded wait" in da2.da2_status_string(5)
