@@ -368,6 +368,57 @@ def run_ours(args, wl):
         dist.destroy_process_group()
 
 
+SWEEP_BUDGETS = [  # skip / 4-bit / 8-bit / 16-bit percentages
+    (95, 0, 0, 5), (90, 0, 0, 10), (85, 0, 0, 15), (80, 0, 0, 20), (70, 0, 0, 30),
+    (90, 0, 10, 0), (85, 0, 15, 0), (80, 0, 20, 0), (70, 0, 30, 0),
+    (90, 10, 0, 0), (85, 15, 0, 0), (80, 20, 0, 0), (70, 30, 0, 0),
+    (85, 0, 7.5, 7.5), (80.7, 14.4, 4.8, 0), (80, 10, 5, 5), (70, 20, 8, 2),
+]
+SWEEP_LAMBDAS = [0.0, 0.25, 0.5, 0.75, 1.0]
+
+
+def run_sweep(args, wl):
+    """Fidelity against latency on one GPU: for a grid of budgets (the Pareto
+    view of the method's allocation) and for lambda at the workload's budget
+    (average-only versus average + max drafting), the call time (CUDA events,
+    median of a few calls) and the relative L2 error of the output against the
+    own dense bf16 attention on the same inputs.  One JSON line per point."""
+    import torch
+    from mixed_precision_block_b200 import da2
+    from mixed_precision_block_b200.synth import make_qkv
+
+    dev = torch.device("cuda", 0)
+    q, k, v = make_qkv(wl, dev)
+    ref = torch.empty_like(q)
+    da2.da2_dense_attention(q, k, v, ref)
+    torch.cuda.synchronize()
+    ref32 = ref.float()
+    ref_norm = float(ref32.norm())
+    out = torch.empty_like(q)
+    points = [(b, wl.lam) for b in SWEEP_BUDGETS] + [(tuple(wl.budget), lam) for lam in SWEEP_LAMBDAS]
+    for budget, lam in points:
+        p = da2.Problem.from_workload(wl, budget=budget, lam=lam)
+        ws = da2.workspace(p, dev)
+        times = []
+        for it in range(1 + args.sweep_calls):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record()
+            da2.da2_prepare(p, q, k, v, ws)
+            da2.da2_draft_rank(p, ws)
+            e[1].record()
+            da2.da2_attention(p, q, k, v, ws, out)
+            e[2].record()
+            torch.cuda.synchronize()
+            if it:
+                times.append((e[0].elapsed_time(e[2]), e[1].elapsed_time(e[2])))
+        times.sort()
+        call_ms, attn_ms = times[len(times) // 2]
+        err = float((out.float() - ref32).norm()) / ref_norm
+        print(json.dumps({"sweep": wl.name, "budget_skip_4_8_16": list(budget), "lambda": lam,
+                          "call_ms": call_ms, "attention_ms": attn_ms, "rel_l2_vs_own_dense": err}), flush=True)
+        del ws
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +434,9 @@ def main():
     ap.add_argument("--cpu-frames", type=int, default=8, help="frames of the CPU-baseline oracle sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="budget and lambda sweep: call time and error against the own dense kernel")
+    ap.add_argument("--sweep-calls", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # fewer warm-up steps would not give a valid number
     from mixed_precision_block_b200.synth import WORKLOADS
@@ -391,7 +445,9 @@ def main():
         wl = wl.with_(lam=args.lam)
     if args.heads is not None:
         wl = wl.with_(H=args.heads)
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args, wl)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_ours(args, wl)

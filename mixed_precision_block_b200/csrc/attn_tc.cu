@@ -238,9 +238,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     else if (u < nu8) { i0 = n16 + 2 * (u - nu16); cnt = min(2, n16 + n8 - i0); }
     else { i0 = n16 + n8 + 2 * (u - nu8); cnt = min(2, n16 + n8 + n4 - i0); }
   };
-  // an INT8 unit's S buffer holds the bias (1.5*2^23 as s32) unless a 16-bit
-  // unit's P was the last thing in it
-  auto i8_biased = [&](int u) { return u < 2 || u - 2 >= nu16; };
+
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q16), 1);
@@ -277,7 +275,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tbase = misc[0];
   if (warp < kSoftmaxWarps) {
-    // S buffers whose first user is an INT8 unit start at the bias
+    // the low-bit accumulator starts at zero
     const uint32_t own = tbase + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * 64;
     bool any = false;
     if (n8 > 0 || n4 > 0) {  // the low-bit accumulator starts at zero
@@ -285,12 +283,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_fill32(own + TM_ACC + 32, 0u);
       any = true;
     }
-    for (int b = 0; b < 2; ++b)
-      if (b >= nu16 && b < nu8) {
-        tmem_fill32(own + TM_S + b * 128, kI8Bias);
-        tmem_fill32(own + TM_S + b * 128 + 32, kI8Bias);
-        any = true;
-      }
     if (any) tmem_wait_st();
   }
   tc_fence_before();
@@ -429,8 +421,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // one (the second holds scale factors), so they wait for the unit
           // before — for the first of them that implies both buffers were read
           // A 16-bit unit's P lives in its S buffer until its P·V completes.
+          // 16-bit and INT8 units leave their P in their S buffer until their
+          // P·V completes
           auto pv_done = [&](int j) {
-            return j < 0 || j >= nu16 || mbar_test(bar(B_P_FREE + (j & 1)), (j >> 1) & 1);
+            return j < 0 || j >= nu8 || mbar_test(bar(B_P_FREE + (j & 1)), (j >> 1) & 1);
           };
           const bool s_free = single ? (sn < 1 || mbar_test(bar(B_S_FREE + ((sn - 1) & 1)), ((sn - 1) >> 1) & 1)) &&
                                            pv_done(sn - 1) && pv_done(sn - 2)
@@ -455,7 +449,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               for (int kk = 0; kk < 4; ++kk)
                 mma_i8(sd, smem_desc(s0 + SM_Q8 + kk * 32, 16, 1024, SW_128),
                        smem_desc(st + kk * 32, 16, 1024, SW_128), id,
-                       (kk > 0 || i8_biased(sn)) ? 1u : 0u);  // onto the bias where it was laid
+                       kk > 0 ? 1u : 0u);
             } else {
               for (int t = 0; t < cnt; ++t) {
                 const uint32_t sfk = tbase + TM_SFK + 8 * t;
@@ -500,8 +494,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               for (int t = 0; t < cnt; ++t) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                  mma_i8(tbase + TM_ACC, smem_desc(pbuf + t * 8192 + kk * 32, 16, 512, SW_64),
-                         smem_desc(st + t * 8192 + kk * 32, 16, 512, SW_64), idx8, 1u);
+                  mma_i8_ta(tbase + TM_ACC, tbase + TM_S + (pn & 1) * 128 + 64 * t + 8 * kk,
+                            smem_desc(st + t * 8192 + kk * 32, 16, 512, SW_64), idx8, 1u);
               }
             } else {
               int i0, cnt;
@@ -778,14 +772,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_ld32(scol + 32, sr + 32);
         tmem_wait_ld();
         if (i8) {
-          // the s32 scores sit on the bias (or are put on it, where a 16-bit
-          // unit used the buffer last): subtracting it gives them exactly
-          // (|S| < 128*127^2 < 2^22)
+          // exact s32 -> fp32 through the mantissa of 1.5*2^23 (|S| < 128*127^2 < 2^22)
           const uint64_t kx2 = f2pack(-kI8BiasF, -kI8BiasF);
-          if (!i8_biased(u)) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) sr[i] += kI8Bias;
-          }
+          for (int i = 0; i < 64; ++i) sr[i] += kI8Bias;
 #pragma unroll
           for (int i = 0; i < 64; i += 2) {
             float a, b;
@@ -888,35 +878,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       if (i8) {
-        // INT8 units alternate two S buffers: re-bias this warp's columns if the
-        // next user is an INT8 unit (the scores are dead now), then release
-        if (u + 2 < nu8) {
-          tmem_fill32(scol, kI8Bias);
-          tmem_fill32(scol + 32, kI8Bias);
-          tmem_wait_st();
-        }
+        // INT8 P codes (four per column, key 4i in the low byte) replace this
+        // warp's scores in TMEM, where the P·V MMA reads them; the buffer goes
+        // back to the score MMAs once that P·V completes
+        if (present) tmem_st16(scol, pw);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_S_FREE + (u & 1)));
       }
-      // the P area and the accumulator are settled once the P·V of the unit
-      // before completed
-      if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
-      tc_fence_after();
-      // a rising reference first folds what the phase holds into O; INT8 also
-      // folds every 256 units, before its s32 sums could overflow
+      // a rising reference first folds what the phase holds into O (INT8 also
+      // every 256 units, before its s32 sums could overflow): the accumulator
+      // is settled once the P·V of the unit before completed.  4-bit P goes
+      // through shared memory, free once that P·V completed too.
       const bool guard = i8 && u > nu16 && ((u - nu16) & 255) == 0;
+      if (!i8 || __any_sync(FULL, raise || guard)) {
+        if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
+        tc_fence_after();
+      }
       fold(raise || guard, i8);
       if (raise) r_lo = r_use;
       l_lo += lp;
-      if (present) {
-        if (i8) {
-          uint8_t* pb = smem + SM_P + half * 8192;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(pb + row * 64 + ((c ^ ((row >> 1) & 3)) * 16)) =
-                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-        } else {
+      if (present && !i8) {
+        {
           uint8_t* pb = smem + SM_P + half * 4096;
 #pragma unroll
           for (int c = 0; c < 2; ++c)
@@ -926,7 +910,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                        (row >> 5) * 4) = sfw;
         }
       }
-      fence_async_smem();
+      if (!i8) fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));

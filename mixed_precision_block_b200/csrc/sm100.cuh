@@ -193,6 +193,14 @@ __device__ __forceinline__ void mma_f16_ta(uint32_t dtmem, uint32_t atmem, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(dtmem), "r"(atmem), "l"(bdesc), "r"(id), "r"(acc));
 }
+// kind::i8 with the A operand (M rows x K bytes, four per 32-bit column) read
+// from tensor memory.
+__device__ __forceinline__ void mma_i8_ta(uint32_t dtmem, uint32_t atmem, uint64_t bdesc, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(dtmem), "r"(atmem), "l"(bdesc), "r"(id), "r"(acc));
+}
 __device__ __forceinline__ void mma_i8(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t id, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"

@@ -244,3 +244,33 @@ def dense_attention(q, k, v):
     s = s - s.max(1, keepdims=True)
     p = np.exp(s)
     return (p @ v) / p.sum(1, keepdims=True)
+
+
+def error_terms(prep, prec_map, d, qblocks, partner=True):
+    """Error decomposition of the method on the given query blocks of one head
+    (DraftAttention2 abstract and reading note, Method overview: sparsity and
+    quantisation are the two approximations; here they are measured apart).
+
+    Returns relative L2 errors against exact dense attention over the real
+    rows of the blocks, all in fp64 (``math`` mode, no output rounding):
+      ``sparse``  exact attention restricted to the retained key blocks,
+      ``quant``   the mixed-precision result minus that exact sparse result,
+      ``total``   the mixed-precision result itself;
+    so total <= sparse + quant (triangle inequality)."""
+    valid = prep["valid"]
+    kept = {BIT16, BIT8, BIT4}
+    num_s = num_q = num_t = den = 0.0
+    for qb in qblocks:
+        row = prec_map[qb]
+        other = partner_of(prec_map, qb) if partner else None
+        mixed = qblock_attention(prep, qb, row, d, "math", other)
+        exact_row = np.where(np.isin(row, list(kept)), BIT16, 0).astype(row.dtype)
+        sparse = qblock_attention(prep, qb, exact_row, d, "math")
+        dense = qblock_attention(prep, qb, np.full_like(row, BIT16), d, "math")
+        rv = valid[qb]
+        num_s += float(((sparse - dense)[rv] ** 2).sum())
+        num_q += float(((mixed - sparse)[rv] ** 2).sum())
+        num_t += float(((mixed - dense)[rv] ** 2).sum())
+        den += float((dense[rv] ** 2).sum())
+    den = max(den, 1e-300)
+    return {"sparse": (num_s / den) ** 0.5, "quant": (num_q / den) ** 0.5, "total": (num_t / den) ** 0.5}

@@ -179,3 +179,25 @@ def test_low_bit_reference_raise_by_hand():
     ph.enter([np.array([[1.0]])])
     ph.enter([np.array([[-np.inf]])])
     assert ph.r[0] == 3.0
+
+
+def _terms(budget, qblocks=None):
+    p, q, k, v = _inputs(budget=budget)
+    r = pipeline.run_head(p, q, k, v, mode="math")
+    qbs = range(p.nb) if qblocks is None else qblocks
+    return attention.error_terms(r["prep"], r["map"], p.d, qbs)
+
+
+def test_error_terms_special_cases():
+    t = _terms((0, 0, 0, 100))  # everything kept at 16 bits: exact
+    assert t["sparse"] < 1e-13 and t["quant"] < 1e-13 and t["total"] < 1e-13
+    t = _terms((100, 0, 0, 0))  # everything skipped: the output is zero
+    assert abs(t["sparse"] - 1.0) < 1e-13 and t["quant"] < 1e-13 and abs(t["total"] - 1.0) < 1e-13
+    t = _terms((0, 0, 100, 0))  # nothing skipped, all INT8: only quantisation error
+    assert t["sparse"] < 1e-13 and abs(t["quant"] - t["total"]) < 1e-13 and 0 < t["quant"] < 0.05
+
+
+def test_error_terms_triangle_and_both_present():
+    t = _terms((40, 20, 20, 20))
+    assert t["total"] <= t["sparse"] + t["quant"] + 1e-12
+    assert t["sparse"] > 0 and t["quant"] > 0
