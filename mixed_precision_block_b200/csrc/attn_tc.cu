@@ -25,27 +25,24 @@
 //           P = exp2(s·log2e/√d − m_ref) rounded to bf16, m_ref an integer
 //           exponent shared by the two warps of a row and raised lazily (O
 //           rescaled in TMEM by a power of two only when the row max grows by
-//           more than 2^8); P goes K-major to shared memory; O += P·V
-//           (kind::f16, V read MN-major from the TMA tile).
-//   Entering the low-bit phases, O moves into registers (each warp its 64
-//   channels), where it stays: the block results of the low-bit phases are
-//   folded into it, and TMEM holds one S buffer and the two block results.
-//   8-bit   S = Q8·[K8_a; K8_b]^T (kind::i8, s32, N128); each warp quantises its
-//           block's P8 = round(255·exp(s − m_blk)) as u8 from its own full
-//           rows, so no statistics cross warps before the MMA;
-//           X_h = P8_h·V8_h^T (kind::i8 u8×s8, s32).  Both warps of a row fold
-//           their 64 channels of X_a and X_b into the register accumulator with
-//           weight exp(m_blk − m); the two warps trade (m_blk, l_blk) through
-//           shared memory one unit late, off the critical path.
+//           more than 2^8).  P replaces the warp's own scores in TMEM and
+//           O += P·V reads it from there as the A operand (kind::f16, V read
+//           MN-major from the TMA tile), so the softmax of a unit never waits
+//           for the P·V of the one before unless O must be rescaled.
+//   Low-bit phases accumulate P·V in TMEM at column 384 (INT8: s32 X8; 4-bit:
+//   fp32 O4) against a power-of-two reference 2^r per row, shared by the two
+//   warps of the row and raised to ceil(unit max) whenever a unit's max
+//   exceeds it; P is quantised relative to 2^r.  Before a raise (INT8 also
+//   every 256 units, ahead of s32 overflow) and at the end of the phase the
+//   accumulator is folded into O with the phase's channel scale (sv/255 or
+//   g/2688) and cleared.
+//   8-bit   S = Q8·[K8_a; K8_b]^T (kind::i8, s32 read back exactly through the
+//           mantissa of 1.5·2^23); codes rint(255 p) as u8 replace the scores
+//           in TMEM; X8 += P8·V8 (kind::i8 u8×s8, A from TMEM).
 //   4-bit   S_h = Q4·K4_h^T (kind::mxf4nvf4, block16 e4m3 scales copied into
-//           TMEM with tcgen05.cp from the scale atoms prep wrote); P
-//           re-quantised to NVFP4 per 16 keys in registers, with its scales
-//           written as an atom; X_h = P4_h·V4_h^T (block-scaled, fp32), folded
-//           in the same way.
-//   The register accumulator is kept divided by the channel scale of the
-//   phase it last took (INT8 sv, NVFP4 g), so a fold is one FMA per element;
-//   crossing a phase boundary re-expresses it in the next phase's scale, and
-//   the epilogue multiplies the last scale back.
+//           TMEM with tcgen05.cp from the scale atoms prep wrote); 2688 p
+//           quantised to NVFP4 per 16 keys in registers, codes and scale atom
+//           to shared memory; O4 += P4·V4 (block-scaled).
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), INT8 codes as 2-D
 // boxes of the workspace.  The epilogue writes O through the same region box
@@ -93,8 +90,8 @@ constexpr uint32_t SM_V = SM_K + kStages * 32768;            // V ring: kStages 
 // per block) at +8192; V slot = V4_a^T | V4_b^T ([128][32 B] SW32, 4 KB each)
 // with one scale atom per block at +8192.
 constexpr uint32_t SL_SF = 8192;
-// P area: 16-bit P_a | P_b (16 KB each).  Low-bit units: P8_a | P8_b (8 KB
-// each) or P4_a | P4_b (4 KB each) at +0 and the P4 scale atoms at +16384.
+// P area (4-bit units only; 16-bit and INT8 P stay in TMEM): P4_a | P4_b
+// (4 KB each) at +0, their scale atoms at +16384.
 constexpr uint32_t SM_P = SM_V + kStages * 32768;
 constexpr uint32_t PO_PSF = 16384;
 // channel scales that fold a low-bit accumulator into O (fp32 [128] each):
@@ -417,12 +414,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             // first 4-bit unit: Q4 must be in shared memory and its scales in TMEM
             f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
           }
-          // 16-bit and INT8 units alternate two S buffers; 4-bit units share
-          // one (the second holds scale factors), so they wait for the unit
-          // before — for the first of them that implies both buffers were read
-          // A 16-bit unit's P lives in its S buffer until its P·V completes.
-          // 16-bit and INT8 units leave their P in their S buffer until their
-          // P·V completes
+          // 16-bit and INT8 units alternate two S buffers and leave their P
+          // there until their P·V completes; 4-bit units share one (the
+          // second holds scale factors), so they wait for the unit before —
+          // for the first of them that implies both buffers were read
           auto pv_done = [&](int j) {
             return j < 0 || j >= nu8 || mbar_test(bar(B_P_FREE + (j & 1)), (j >> 1) & 1);
           };
