@@ -477,12 +477,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_mp_kernel(Geom g, AttnAr
     if (ux1 != -INFINITY && (r[1] == -INFINITY || ux1 > r[1])) r[1] = ceilf(ux1);
   };
   const int tq = lane & 3;
+  // the phases share the softmax statistics: the low-bit reference starts from
+  // the 16-bit phase's, ceil of the running row maximum (-inf if it had no
+  // block), and carries on from the 8-bit phase into the 4-bit one
+  float r[2] = {m[0], m[1]};
   // ---------------- phase 8
   if (cnt.y > 0) {
     load_bytes_swz<D>(s0 + SL::Q, reinterpret_cast<const uint8_t*>(A.q_i8) + row_lin * 64 * D, 64);
     for (int c = threadIdx.x; c < D; c += kAttnThreads) vs[c] = A.v_s8[(size_t)bh * D + c];
     const float sq = A.q_s8[row_lin];
-    float r[2] = {-INFINITY, -INFINITY};
     const uint32_t* it8 = items + pc.x;
     for (int i = 0; i < pc.y; i += 2) {
       int kbs[2];
@@ -516,7 +519,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_mp_kernel(Geom g, AttnAr
   if (cnt.z > 0) {
     dequant_f4_tile<D>(smem + SL::Q, A.q_f4 + row_lin * 64 * (D / 2), A.q_sf4 + row_lin * SL::KSF, 64);
     for (int c = threadIdx.x; c < D; c += kAttnThreads) vs[c] = A.v_g4[(size_t)bh * D + c];
-    float r[2] = {-INFINITY, -INFINITY};
     const uint32_t* it4 = items + pc.x + pc.y;
     for (int i = 0; i < pc.z; i += 2) {
       int kbs[2];

@@ -137,7 +137,6 @@ struct TcArgs {
   const uint8_t* v_sf4;
   int* status;
   int npairs;
-  int dense;  // every key block in the 16-bit phase; no item lists are read
 };
 
 __device__ __forceinline__ void raise_timeout(int* status) { atomicOr(status, 1); }
@@ -191,6 +190,9 @@ __device__ __forceinline__ unsigned long long key_mask(const Geom& g, int kb) {
   return m;
 }
 
+// kDense: every key block in the 16-bit phase, no item lists read (a separate
+// instantiation, so that the sparse kernel carries none of it)
+template <bool kDense>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -207,13 +209,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qa = 2 * pair, qb = (2 * pair + 1 < g.nb) ? 2 * pair + 1 : -1;
   const size_t prow = (size_t)bh * A.npairs + pair;
-  const int4 pc = A.dense ? make_int4(g.nb, 0, 0, 0) : *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
+  const int4 pc = kDense ? make_int4(g.nb, 0, 0, 0) : *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
   const int n16 = pc.x, n8 = pc.y, n4 = pc.z;
-  const uint32_t* items = A.dense ? nullptr : A.plist + prow * (size_t)(2 * g.nb);
+  const uint32_t* items = kDense ? nullptr : A.plist + prow * (size_t)(2 * g.nb);
   // entry i of the pair's list; in dense mode key block i, kept by both query
   // blocks, flagged full unless it holds the ragged tail
   auto item_at = [&](int i) -> uint32_t {
-    if (!A.dense) return items[i];
+    if (!kDense) return items[i];
     return (uint32_t)i | (1u << 16) | ((2 * pair + 1 < g.nb ? 1u : 0u) << 17) |
            ((uint32_t)((i + 1) * 64 <= g.N) << 20);
   };
@@ -261,7 +263,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(s0 + SM_MISC, 512);
-  if (threadIdx.x < kD && !A.dense) {
+  if (threadIdx.x < kD && !kDense) {
     const float sv = A.v_s8[(size_t)bh * kD + threadIdx.x], gv = A.v_g4[(size_t)bh * kD + threadIdx.x];
     float* vsc = reinterpret_cast<float*>(smem + SM_VS);
     vsc[VS_SV255 / 4 + threadIdx.x] = sv / 255.0f;
@@ -543,6 +545,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return v < 0 || mbar_wait(bar(B_P_FREE + (v & 1)), (uint32_t)(v >> 1) & 1u);
     };
     float m16 = -INFINITY, l16 = 0.f;  // 16-bit phase: O in TMEM, integer reference
+    float x_run = -INFINITY;            // running row max (log2 units) over every unit so far
     bool ok = true;
     {  // O starts at zero (this warp's 64 columns)
       uint32_t z[32];
@@ -608,6 +611,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         sk_next = sk_for(u + 1, e_next);  // the entry has arrived by now; the scale has a unit's time
         mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * sl2;  // unit row max, log2 units
         const bool row_live = mx != -INFINITY;  // the row is a member of some block of the unit
+        x_run = fmaxf(x_run, mx);
         const bool need = row_live && (mx > m16 + kRescaleThreshold || m16 == -INFINITY);
         const bool need_o = need && m16 != -INFINITY;
         const float a = need_o ? ldexpf(1.0f, (int)(m16 - ceilf(mx))) : 1.0f;
@@ -667,11 +671,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // row, shared by the two warps of the row; P is quantised relative to 2^r.
     // When a unit's row maximum exceeds r, the accumulator is first folded
     // into O with the phase's channel scale (sv/255 or g/2688) and cleared;
-    // so is it at the end of the phase.  l8/l4 are this warp's partial sums
+    // so is it at the end of the phase.  l_lo is this warp's partial sum of p
     // against the same reference.
     const float* chs8 = reinterpret_cast<const float*>(smem + SM_VS + VS_SV255);
     const float* chs4 = reinterpret_cast<const float*>(smem + SM_VS + VS_G2688);
-    float r_lo = -INFINITY, l_lo = 0.f;
+    // the phases share the softmax statistics: a low-bit phase starts from the
+    // ceiling of the running maximum of everything before it
+    float r_lo = ceilf(x_run), l_lo = 0.f;
     // fold the phase accumulator (this warp's 64 channels) into O for the
     // lanes in `sel`; O's reference becomes max(m16, r_lo) for them
     auto fold = [&](bool sel, bool i8) {
@@ -715,8 +721,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // P·V completed; the columns then start the 4-bit accumulator at zero
         if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
         tc_fence_after();
-        fold(true, true);
-        r_lo = -INFINITY;
+        fold(true, true);  // the reference carries on into the 4-bit phase
       }
       int i0, cnt;
       unit_items(u, i0, cnt);
@@ -1119,11 +1124,10 @@ cudaError_t launch_dense_tc(int B, int H, int N, const void* q, const void* k, c
   TcArgs A{};
   A.status = status;
   A.npairs = (g.nb + 1) / 2;
-  A.dense = 1;
-  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   // the low-bit tensor maps are never used in dense mode
-  attn_tc_kernel<<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq, tk, tv, tq, tk, tv, g, A);
+  attn_tc_kernel<true><<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq, tk, tv, tq, tk, tv, g, A);
   return cudaGetLastError();
 }
 
@@ -1161,10 +1165,10 @@ cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, c
   A.v_sf4 = at<uint8_t>(ws, L, R_V_SF4);
   A.status = status;
   A.npairs = (g.nb + 1) / 2;
-  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq8, tk8, tv8, tq4, tk4, tv4,
-                                                                      g, A);
+  attn_tc_kernel<false><<<dim3(A.npairs, g.BH), kThreads, kSmemBytes, st>>>(tq, tk, tv, to, tq8, tk8, tv8, tq4, tk4,
+                                                                             tv4, g, A);
   return cudaGetLastError();
 }
 

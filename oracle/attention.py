@@ -8,9 +8,10 @@ outputs are written back and merged.  Skipped pairs contribute nothing.
 
 This module follows that structure literally, per query block, in fp64:
 phase 16, then phase 8, then phase 4, one online-softmax state (m, l, O)
-carried across all of them; each low-bit phase accumulates against its own
-power-of-two reference and is folded into that state, with its channel
-scales, at the phase boundary.
+carried across all of them; each low-bit phase accumulates in its own
+accumulator against a power-of-two reference that starts from the running
+maximum of the phases before it, and is folded into that state, with its
+channel scales, at the phase boundary.
 
 Readings adopted (the pages leave these open):
 
@@ -23,15 +24,18 @@ Readings adopted (the pages leave these open):
   consecutive pairs.  A unit's blocks that this query block does not retain
   contribute nothing to its rows.
 * P in the 8-bit and 4-bit phases is quantised relative to a running power of
-  two 2^r per row and phase (r an integer, log2 units): before a unit, if the
-  unit's row maximum x_max (of s·log2 e over its retained keys) exceeds r, r
-  becomes ceil(x_max), and what the phase accumulated so far is scaled by
-  2^(r_old - r).  So p = 2^(x - r) is in (0, 1]:
+  two 2^r per row (r an integer, log2 units).  The phases share the softmax
+  statistics, so a low-bit phase starts from r = ceil(x_run), x_run the row's
+  running maximum of s·log2 e over every unit of the phases before it (-inf
+  if there was none).  Before a unit, if the unit's row maximum x_max (over
+  its retained keys) exceeds r, r becomes ceil(x_max), and what the phase
+  accumulated so far is scaled by 2^(r_old - r).  So p = 2^(x - r) is in
+  (0, 1]:
   8-bit code = round(255 p) as an unsigned byte (scale 1/255);
   4-bit = NVFP4, over 16 consecutive keys of the row, of 2688 p (2688 = 6·448
   puts the largest p at the top of the e2m1 x e4m3 range), dequantised and
-  divided by 2688 again.  Each phase accumulates its P·V against its own
-  reference; the phases' results meet, with the channel scales, at the end.
+  divided by 2688 again.  Each phase accumulates its P·V in its own
+  accumulator; the phases' results meet, with the channel scales, at the end.
 * the softmax denominator l sums the unquantised exp(s - m) over every retained
   real key of every phase.
 * 16-bit phase, ``emulate`` mode: P is rounded to bf16 relative to a power of
@@ -97,8 +101,8 @@ class _LowBitPhase:
     """A low-bit phase's P·V accumulator and sum against a running power of two
     2^r per row (r an integer, log2 units; -inf before the first score)."""
 
-    def __init__(self, rows, d):
-        self.r = np.full(rows, -np.inf)
+    def __init__(self, rows, d, r0=None):
+        self.r = np.full(rows, -np.inf) if r0 is None else np.array(r0, dtype=np.float64)
         self.l = np.zeros(rows)
         self.acc = np.zeros((rows, d))
 
@@ -108,6 +112,7 @@ class _LowBitPhase:
         where that max exceeds r, rescale what is accumulated, add the
         unquantised p to l and return each block's p = 2^(x - r)."""
         x_max = np.max(np.stack([x.max(1) for x in xs]), axis=0)
+        self.x_max = x_max
         up = np.isfinite(x_max) & (x_max > self.r)
         r_new = np.where(up, np.ceil(np.where(up, x_max, 0.0)), self.r)
         had = np.isfinite(self.r)
@@ -140,23 +145,27 @@ def _exp_rel(s, m):
     return np.where(ok, np.exp(np.where(ok, s - np.where(np.isfinite(m), m, 0)[:, None], 0)), 0.0)
 
 
-def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None):
+def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None, trace=None):
     """Output rows [S, d] of query block ``qb`` of one head.
 
     ``prep``: dict from ``prep.prepare_head``; ``prec_row``: uint8 [nb] precision
     of each key block for this query block (16, 8, 4, 0); ``partner_row``: the
     same for the other query block of its pair (qb ^ 1), None if there is none.
-    The partner only decides how the low-bit phases group key blocks into units."""
+    The partner only decides how the low-bit phases group key blocks into units.
+    ``trace``: a dict that receives each low-bit phase's starting reference
+    (``r0_8``, ``r0_4``, per row)."""
     S = prep["q_blocks"].shape[1]
     valid = prep["valid"]
     inv_sqrt_d = 1.0 / np.sqrt(d)
     st = _State(S, d)
+    x_run = np.full(S, -np.inf)  # running row max of s·log2 e, every phase so far
 
     # phase 16: bf16 operands, online softmax across blocks
     q = prep["q_blocks"][qb]
     for kb in np.nonzero(prec_row == BIT16)[0]:
         s = (q @ prep["k_blocks"][kb].T) * inv_sqrt_d
         s = np.where(valid[kb][None, :], s, -np.inf)
+        x_run = np.maximum(x_run, _row_max(s) * LOG2E)
         m_new = np.maximum(st.m, _row_max(s))
         if mode == "emulate":
             # P is rounded in bf16 relative to 2^ceil(m_run log2 e), then brought
@@ -177,7 +186,9 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None):
     # phase 8: INT8 Q/K codes with block scales, u8 P, INT8 V with channel scales
     qi = prep["q_i8"][qb].astype(np.float64)
     sq = prep["q_s8"][qb]
-    ph = _LowBitPhase(S, d)
+    ph = _LowBitPhase(S, d, np.ceil(x_run))
+    if trace is not None:
+        trace["r0_8"] = ph.r.copy()
     for unit in phase_units(prec_row, partner_row, BIT8):
         xs = []
         for kb in unit:
@@ -188,11 +199,14 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None):
         for kb, p in zip(unit, ph.enter(xs)):
             code = np.rint(255.0 * p)
             ph.acc += code @ prep["v_i8"][kb].astype(np.float64).T  # exact integers
+        x_run = np.maximum(x_run, ph.x_max)
     ph.fold_into(st, prep["v_s8"][None, :] / 255.0)
 
     # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks of 2688 p), NVFP4 V
     qd = F.nvfp4_dequantize(prep["q_f4"][qb], prep["q_sf4"][qb])
-    ph = _LowBitPhase(S, d)
+    ph = _LowBitPhase(S, d, np.ceil(x_run))
+    if trace is not None:
+        trace["r0_4"] = ph.r.copy()
     for unit in phase_units(prec_row, partner_row, BIT4):
         xs = []
         for kb in unit:

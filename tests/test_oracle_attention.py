@@ -201,3 +201,44 @@ def test_error_terms_triangle_and_both_present():
     t = _terms((40, 20, 20, 20))
     assert t["total"] <= t["sparse"] + t["quant"] + 1e-12
     assert t["sparse"] > 0 and t["quant"] > 0
+
+
+def _two_level_head(d=64):
+    """One frame of 8x24 tokens = three full 8x8 regions (key blocks 0, 1, 2).
+    Every query is 8 e_0; keys of block 0 are 8 e_0 (score 64/sqrt(64) = 8,
+    x = 8 log2 e = 11.54 in log2 units), keys of blocks 1 and 2 are 0 (score
+    0).  V rows are small integers, exact in every format's scale."""
+    p = Problem(1, 1, 1, 8, 24, d, 0.5, (0, 0, 0, 100))
+    tab = geometry.block_tokens(p)
+    q = np.zeros((p.N, d))
+    q[:, 0] = 8.0
+    k = np.zeros((p.N, d))
+    k[tab[0], 0] = 8.0
+    v = np.random.default_rng(3).integers(-3, 4, size=(p.N, d)).astype(np.float64)
+    return p, prep.prepare_head(p, q, k, v), v, tab
+
+
+def test_low_bit_phase_starts_from_the_shared_running_max():
+    # block 0 at 16 bits sets the running max x = 11.54; the 8-bit phase then
+    # starts from r = ceil(11.54) = 12, so block 1's p = 2^(0 - 12) gives code
+    # rint(255 / 4096) = 0: block 1 adds its unquantised mass 64 e^-8 to the
+    # denominator and nothing to the numerator.  (A phase that restarted its
+    # reference would take r = 0 and code 255 instead.)
+    p, pr, v, tab = _two_level_head()
+    row = np.array([16, 8, 0], dtype=np.uint8)
+    tr = {}
+    out = attention.qblock_attention(pr, 0, row, p.d, "math", None, trace=tr)
+    np.testing.assert_array_equal(tr["r0_8"], np.full(64, 12.0))
+    want = v[tab[0]].mean(0) / (1.0 + np.exp(-8.0))
+    np.testing.assert_allclose(out, np.broadcast_to(want, out.shape), rtol=1e-12, atol=1e-15)
+
+
+def test_four_bit_phase_continues_the_reference_of_the_eight_bit_phase():
+    # block 0 at 8 bits (INT8 codes 127 and scale 8/127 reproduce the score 8
+    # exactly) and block 2 at 4 bits: the 4-bit phase starts from ceil(11.54) = 12
+    p, pr, v, tab = _two_level_head()
+    row = np.array([8, 0, 4], dtype=np.uint8)
+    tr = {}
+    attention.qblock_attention(pr, 0, row, p.d, "math", None, trace=tr)
+    assert np.all(np.isneginf(tr["r0_8"]))  # nothing before the 8-bit phase
+    np.testing.assert_array_equal(tr["r0_4"], np.full(64, 12.0))
