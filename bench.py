@@ -51,6 +51,16 @@ def phase_flops(wl, info):
     return {16: per_pair * info.n16 * bh, 8: per_pair * info.n8 * bh, 4: per_pair * info.n4 * bh}
 
 
+# XU-pipe work per retained 64x64 block pair in the attention kernel: one ex2
+# per score, plus the F2FP conversions that issue to the same pipe (16-bit: one
+# bf16x2 per two probabilities; 4-bit: one e2m1x2 per two and one e4m3 per
+# sixteen; INT8 codes are formed on the FMA pipe).  The pipe retires 16 lanes
+# per clock per SM (4,096 ex2 per sub-partition took ~1,030 cycles in a probe).
+XU_PER_PAIR = {16: 64 * 64 * 1.5, 8: 64 * 64 * 1.0, 4: 64 * 64 * (1.5 + 1.0 / 16)}
+XU_LANES_PER_CLK_SM = 16
+SMS = 148
+
+
 def launches_per_call(info, d):
     """Kernels this library launches per call (its own kernels only)."""
     v = 2 if (info.n8 or info.n4) else 0  # v_amax + pack_v
@@ -298,16 +308,14 @@ def run_ours(args, wl):
     # end to end through host buffers: pinned H2D of Q/K/V, the call, D2H of O
     e2e = None
     if not args.no_e2e:
+        # the public host-buffer call: chunks of heads, the copies of one chunk
+        # overlapped with the kernels of another, synchronous
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        hbuf = da2.host_buffer(p, args.e2e_chunk, dev)
 
         def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            da2.attention(p, dq, dk, dv, ws, out, st)
-            hout.copy_(out, non_blocking=True)
+            da2.da2_forward_host(p, hq, hk, hv, hout, hbuf, args.e2e_chunk, st)
 
         with torch.cuda.stream(st):
             e2e_step()
@@ -324,8 +332,9 @@ def run_ours(args, wl):
             e_ms = float(t.item())
         nbytes = q.numel() * q.element_size()
         e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
-        del hq, hk, hv, hout, dq, dk, dv
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "call": f"da2_forward_host on pinned host tensors, chunks of {args.e2e_chunk} (batch, head) slices"}
+        del hq, hk, hv, hout, hbuf
 
     pk, pk_kind = peaks()
     sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -338,6 +347,26 @@ def run_ours(args, wl):
     kname, ksrc = roofline_kernel(wl)
     traffic = traffic_record(kname, os.path.join(ROOT, "mixed_precision_block_b200", "csrc", ksrc), wl.name)
     clocks = clk.summary()
+    # the softmax's XU floor beside the tensor floor; the larger one bounds the kernel
+    bh = wl.B * wl.H
+    xu_ops = bh * (info.n16 * XU_PER_PAIR[16] + info.n8 * XU_PER_PAIR[8] + info.n4 * XU_PER_PAIR[4])
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    xu_peak = XU_LANES_PER_CLK_SM * SMS * mhz * 1e6  # ops/s
+    floors_ms = {"tensor": t_roof_s * 1e3, "xu": xu_ops / xu_peak * 1e3}
+    if floors_ms["xu"] > floors_ms["tensor"]:
+        roof = {"bound": "alu", "kernel": kname, "achieved": xu_ops / (attn_ms * 1e-3) / 1e9,
+                "peak": xu_peak / 1e9, "unit": "Gop/s", "frac": floors_ms["xu"] / attn_ms,
+                "traffic": traffic,
+                "peak_note": f"XU pipe (ex2 + F2FP conversions), {XU_LANES_PER_CLK_SM} lanes/clk/SM x {SMS} SMs "
+                             f"at {mhz:.0f} MHz; tensor floor {floors_ms['tensor']:.2f} ms is lower"}
+    else:
+        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved,
+                "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
+                "traffic": traffic,
+                "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
+                             f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
+                             f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"}
+    roof["floors_ms"] = floors_ms
 
     if rank == 0:
         cpu = None
@@ -353,12 +382,7 @@ def run_ours(args, wl):
             "dense_bf16": None if dense_ms is None else {
                 "ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
                 "speedup_of_sparse_call": dense_ms / ms},
-            "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved,
-                         "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
-                         "traffic": traffic,
-                         "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
-                                      f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
-                                      f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"},
+            "roofline": roof,
             "e2e": e2e, "gpu_launches": launches_per_call(info, wl.d) * args.steps, "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -430,6 +454,7 @@ def main():
     ap.add_argument("--heads", type=int, default=None, help="run only this many heads (profiling captures)")
     ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunk", type=int, default=3, help="(batch, head) slices per chunk of the host-buffer call")
     ap.add_argument("--ref-frames", type=int, default=2, help="frames per CPU oracle sample (reference arm)")
     ap.add_argument("--cpu-frames", type=int, default=8, help="frames of the CPU-baseline oracle sample")
     ap.add_argument("--no-e2e", action="store_true")

@@ -201,6 +201,32 @@ int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, ui
  * on the pages: it reports this implementation's own wait bounds. */
 int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void* stream);
 
+/* Host-buffer form of the whole path (da2_prepare, da2_draft_rank and
+ * da2_attention) for callers whose Q/K/V and output live in host memory.
+ * The (batch, head) slices run in chunks of heads_per_chunk, each chunk a
+ * problem of its own (every stage is per head: DraftAttention2 reading note,
+ * Method overview bullets 1-4, one ranking per head); two sets of device
+ * buffers alternate so that the host<->device copies of one chunk overlap the
+ * kernels of another.  No counterpart on the pages.
+ *
+ * da2_host_bytes: bytes of the device buffer da2_forward_host needs for this
+ * problem and chunk size (two sets of chunk Q, K, V, output and workspace,
+ * plus one status word per chunk).
+ *
+ * da2_forward_host: q, k, v: host [B,H,T*Hh*Ww,d] bf16, read; out: host
+ * [B,H,N,d] bf16, written in token order.  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister) for the copies to run asynchronously;
+ * pageable memory is correct but serialises them.  dev: caller-owned device
+ * buffer of at least da2_host_bytes bytes, 256-byte aligned.  stream: work
+ * already queued on it runs first; the call creates two copy streams of its
+ * own for its duration.  Synchronous: returns once the output is on the host.
+ * Returns DA2_OK, DA2_ERR_ARG / _UNSUPPORTED (problem, as da2_plan),
+ * DA2_ERR_WORKSPACE (dev missing, misaligned or too small), DA2_ERR_TIMEOUT
+ * (a bounded wait in some chunk's attention kernel expired) or DA2_ERR_CUDA. */
+int da2_host_bytes(const da2_problem* p, int heads_per_chunk, size_t* bytes);
+int da2_forward_host(const da2_problem* p, const void* q, const void* k, const void* v, void* out,
+                     void* dev, size_t dev_bytes, int heads_per_chunk, void* stream);
+
 const char* da2_status_string(int status);
 
 #ifdef __cplusplus

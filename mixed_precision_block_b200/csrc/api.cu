@@ -70,6 +70,44 @@ bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
 
+// Host-buffer path: the (batch, head) slices run in chunks of G, each chunk a
+// problem of its own (B = 1, H = chunk size; every stage is per head).  Two
+// sets of device buffers alternate so that one chunk's copies overlap the
+// other's kernels.
+struct HostPlan {
+  da2_problem pc;   // chunk problem, H = G
+  int BH, G, nchunks;
+  size_t slice;     // bytes of one (b, h) slice of Q, K, V or O (bf16)
+  size_t chunk;     // bytes of one chunk of one tensor, 256-aligned
+  size_t ws;        // workspace bytes of a full chunk
+  size_t set;       // q, k, v, out and workspace of one set
+  size_t status;    // per-chunk status words after the two sets
+  size_t status_off;  // the status word's offset in a chunk workspace
+};
+
+int host_plan(const da2_problem* p, int heads_per_chunk, HostPlan* hp) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (heads_per_chunk <= 0) return DA2_ERR_ARG;
+  hp->BH = g.BH;
+  hp->G = heads_per_chunk < g.BH ? heads_per_chunk : g.BH;
+  hp->nchunks = (g.BH + hp->G - 1) / hp->G;
+  hp->pc = *p;
+  hp->pc.B = 1;
+  hp->pc.H = hp->G;
+  Geom gc;
+  if ((rc = make_geom(&hp->pc, &gc))) return rc;
+  hp->slice = (size_t)g.N * g.d * 2;
+  hp->chunk = (hp->slice * hp->G + 255) & ~(size_t)255;
+  const Layout Lc = make_layout(gc);
+  hp->ws = Lc.total;
+  hp->status_off = Lc.off[R_STATUS];
+  hp->set = 4 * hp->chunk + hp->ws;
+  hp->status = ((size_t)hp->nchunks * sizeof(int) + 255) & ~(size_t)255;
+  return DA2_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -192,6 +230,87 @@ int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
   return word ? DA2_ERR_TIMEOUT : DA2_OK;
+}
+
+int da2_host_bytes(const da2_problem* p, int heads_per_chunk, size_t* bytes) {
+  HostPlan hp;
+  int rc = host_plan(p, heads_per_chunk, &hp);
+  if (rc) return rc;
+  if (!bytes) return DA2_ERR_ARG;
+  *bytes = 2 * hp.set + hp.status;
+  return DA2_OK;
+}
+
+int da2_forward_host(const da2_problem* p, const void* q, const void* k, const void* v, void* out,
+                     void* dev, size_t dev_bytes, int heads_per_chunk, void* stream) {
+  HostPlan hp;
+  int rc = host_plan(p, heads_per_chunk, &hp);
+  if (rc) return rc;
+  if (!q || !k || !v || !out) return DA2_ERR_ARG;
+  if (!dev || ((uintptr_t)dev & 255) != 0 || dev_bytes < 2 * hp.set + hp.status) return DA2_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+  cudaStream_t cs = (cudaStream_t)stream, hs = nullptr, ds = nullptr;
+  cudaEvent_t start = nullptr, ev[3][2] = {};  // [copies in, kernels, copy out][set]
+  cudaError_t e = cudaStreamCreateWithFlags(&hs, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ds, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+  for (int i = 0; i < 3; ++i)
+    for (int s = 0; s < 2; ++s)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev[i][s], cudaEventDisableTiming);
+  // the copy streams start after whatever the caller queued on its stream
+  if (e == cudaSuccess) e = cudaEventRecord(start, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs, start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, start, 0);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(dev) + 2 * hp.set);
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, hp.status, cs);
+  for (int c = 0; c < hp.nchunks && e == cudaSuccess && rc == DA2_OK; ++c) {
+    const int s = c & 1, h0 = c * hp.G, gh = (hp.BH - h0) < hp.G ? (hp.BH - h0) : hp.G;
+    char* base = static_cast<char*>(dev) + s * hp.set;
+    char *dq = base, *dk = base + hp.chunk, *dv = base + 2 * hp.chunk, *dout = base + 3 * hp.chunk;
+    char* ws = base + 4 * hp.chunk;
+    const size_t off = (size_t)h0 * hp.slice, nbytes = (size_t)gh * hp.slice;
+    // copies in, once the kernels of the chunk two back released this set
+    if (c >= 2) e = cudaStreamWaitEvent(hs, ev[1][s], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dq, static_cast<const char*>(q) + off, nbytes, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dk, static_cast<const char*>(k) + off, nbytes, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dv, static_cast<const char*>(v) + off, nbytes, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[0][s], hs);
+    // the kernels, once the copies are in and the output of the chunk two back is out
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev[0][s], 0);
+    if (e == cudaSuccess && c >= 2) e = cudaStreamWaitEvent(cs, ev[2][s], 0);
+    if (e != cudaSuccess) break;
+    da2_problem pcc = hp.pc;
+    pcc.H = gh;
+    if ((rc = da2_prepare(&pcc, dq, dk, dv, ws, hp.ws, cs)) == DA2_OK &&
+        (rc = da2_draft_rank(&pcc, ws, hp.ws, cs)) == DA2_OK)
+      rc = da2_attention(&pcc, dq, dk, dv, ws, hp.ws, dout, cs);
+    if (rc != DA2_OK) break;
+    // the chunk's bounded-wait status (the next use of the workspace clears it)
+    e = cudaMemcpyAsync(status + c, ws + hp.status_off, sizeof(int), cudaMemcpyDeviceToDevice, cs);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1][s], cs);
+    // copy out
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev[1][s], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(static_cast<char*>(out) + off, dout, nbytes, cudaMemcpyDeviceToHost, ds);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2][s], ds);
+  }
+  // the call returns with the output on the host
+  const cudaError_t e1 = cudaStreamSynchronize(hs), e2 = cudaStreamSynchronize(cs), e3 = cudaStreamSynchronize(ds);
+  if (e == cudaSuccess) e = e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3);
+  if (e == cudaSuccess && rc == DA2_OK) {
+    for (int c = 0; c < hp.nchunks && e == cudaSuccess; ++c) {
+      int word = 0;
+      e = cudaMemcpy(&word, status + c, sizeof(int), cudaMemcpyDeviceToHost);
+      if (word) rc = DA2_ERR_TIMEOUT;
+    }
+  }
+  for (int i = 0; i < 3; ++i)
+    for (int s = 0; s < 2; ++s)
+      if (ev[i][s]) cudaEventDestroy(ev[i][s]);
+  if (start) cudaEventDestroy(start);
+  if (hs) cudaStreamDestroy(hs);
+  if (ds) cudaStreamDestroy(ds);
+  if (rc != DA2_OK) return rc;
+  return cuda_status(e);
 }
 
 const char* da2_status_string(int s) {

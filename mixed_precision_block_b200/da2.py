@@ -27,7 +27,7 @@ VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_
          "SCORES", "MAP", "LISTS", "COUNTS", "STATUS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
            "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_check_status",
-           "da2_status_string"]
+           "da2_host_bytes", "da2_forward_host", "da2_status_string"]
 NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
 
 
@@ -67,6 +67,8 @@ _lib.da2_dense_attention.argtypes = [ctypes.c_int] * 4 + [_vp] * 5
 _lib.da2_debug_view.argtypes = [_P, _vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]
 _lib.da2_rank_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
 _lib.da2_check_status.argtypes = [_P, _vp, _sz, _vp]
+_lib.da2_host_bytes.argtypes = [_P, ctypes.c_int, ctypes.POINTER(_sz)]
+_lib.da2_forward_host.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _sz, ctypes.c_int, _vp]
 _lib.da2_status_string.argtypes = [ctypes.c_int]
 _lib.da2_status_string.restype = ctypes.c_char_p
 for _f in EXPORTS[:-1]:
@@ -143,6 +145,32 @@ def da2_check_status(p, ws, stream=None):
     """Synchronise `stream` and return the status of the last attention on `ws`
     (0, or DA2_ERR_TIMEOUT = 5 if a bounded wait in the kernel expired)."""
     return _lib.da2_check_status(ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream, ws))
+
+
+def da2_host_bytes(p, heads_per_chunk):
+    n = _sz()
+    _check("da2_host_bytes", _lib.da2_host_bytes(ctypes.byref(p), int(heads_per_chunk), ctypes.byref(n)))
+    return n.value
+
+
+def host_buffer(p, heads_per_chunk, device="cuda") -> torch.Tensor:
+    """Caller-owned device buffer (uint8) for `da2_forward_host`."""
+    buf = torch.empty(da2_host_bytes(p, heads_per_chunk), dtype=torch.uint8, device=device)
+    assert buf.data_ptr() % 256 == 0
+    return buf
+
+
+def da2_forward_host(p, q, k, v, out, dev, heads_per_chunk, stream=None):
+    """The whole call on host (ideally pinned) bf16 tensors: chunks of
+    `heads_per_chunk` (batch, head) slices, copies overlapped with kernels;
+    returns once `out` holds the result."""
+    for t in (q, k, v, out):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("da2_forward_host takes contiguous bf16 host tensors")
+    _check("da2_forward_host", _lib.da2_forward_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                     _ptr(dev), dev.numel(), int(heads_per_chunk),
+                                                     _stream(stream, dev)))
+    return out
 
 
 def da2_dense_attention(q, k, v, out, stream=None):

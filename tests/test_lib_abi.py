@@ -111,3 +111,29 @@ def test_status_strings(da2):
     assert "workspace" in da2.da2_status_string(3)
     assert da2.da2_status_string(99) == "unknown status"
     assert "bounded wait" in da2.da2_status_string(5)
+
+
+def test_host_path_sizes_and_argument_checks(da2):
+    # two sets of (Q, K, V, O chunk + chunk workspace) plus one status word per
+    # chunk; a chunk of G heads is the same problem with B = 1, H = G
+    wl = WORKLOADS["mid"]
+    p = da2.Problem.from_workload(wl)
+    info = da2.da2_plan(p)
+    for G in (1, 5, 12, 40):
+        Gc = min(G, wl.B * wl.H)
+        pc = da2.Problem.from_workload(wl, B=1, H=Gc)
+        chunk = -(-info.N * wl.d * 2 * Gc // 256) * 256
+        nchunks = -(-(wl.B * wl.H) // Gc)
+        status = -(-nchunks * 4 // 256) * 256
+        want = 2 * (4 * chunk + da2.da2_plan(pc).ws_bytes) + status
+        assert da2.da2_host_bytes(p, G) == want
+    with pytest.raises(da2.Da2Error) as e:
+        da2.da2_host_bytes(p, 0)
+    assert e.value.code == da2.DA2_ERR_ARG
+    # a missing device buffer is refused before any CUDA call
+    null = ctypes.c_void_p(None)
+    host = ctypes.c_void_p(16)
+    rc = da2._lib.da2_forward_host(ctypes.byref(p), host, host, host, host, null, 0, 4, null)
+    assert rc == da2.DA2_ERR_WORKSPACE
+    rc = da2._lib.da2_forward_host(ctypes.byref(p), null, host, host, host, null, 0, 4, null)
+    assert rc == da2.DA2_ERR_ARG
