@@ -61,6 +61,22 @@ XU_LANES_PER_CLK_SM = 16
 SMS = 148
 
 
+def max_over_ranks(x, device, world):
+    """The largest of the ranks' values; every rank takes the same collective."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, flops_per_rank, ms):
+    """Whole-job throughput (TFLOP/s): every rank's work over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def launches_per_call(info, d):
     """Kernels this library launches per call (its own kernels only)."""
     v = 2 if (info.n8 or info.n4) else 0  # v_amax + pack_v
@@ -284,11 +300,8 @@ def run_ours(args, wl):
     barrier()
     ms = t_start.elapsed_time(t_end) / args.steps
     stage = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * flops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(ms, dev, world)
+    value = whole_job_value(world, flops, ms)
 
     # own dense bf16 kernel on the same inputs
     dense_ms = None
@@ -326,12 +339,9 @@ def run_ours(args, wl):
             a1.record(st)
         torch.cuda.synchronize(dev)
         e_ms = a0.elapsed_time(a1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, dev, world)
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": whole_job_value(world, flops, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "call": f"da2_forward_host on pinned host tensors, chunks of {args.e2e_chunk} (batch, head) slices"}
         del hq, hk, hv, hout, hbuf
