@@ -772,30 +772,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_ld32(scol + 32, sr + 32);
         tmem_wait_ld();
         if (i8) {
-          // exact s32 -> fp32 through the mantissa of 1.5*2^23 (|S| < 128*127^2 < 2^22)
-          const uint64_t kx2 = f2pack(-kI8BiasF, -kI8BiasF);
+          // the row max on the integer scores (padding keys at INT_MIN); their
+          // conversion to fp32 waits until after the max exchange
+          if (!full) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) sr[i] += kI8Bias;
-#pragma unroll
-          for (int i = 0; i < 64; i += 2) {
-            float a, b;
-            f2unpack(f2add(f2pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), kx2), a, b);
-            sr[i] = __float_as_uint(a);
-            sr[i + 1] = __float_as_uint(b);
+            for (int i = 0; i < 64; ++i)
+              if (!((vm >> i) & 1ull)) sr[i] = 0x80000000u;
           }
+          int m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+#pragma unroll
+          for (int i = 0; i < 64; i += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              m4[q] = max(m4[q], max((int)sr[i + 2 * q], (int)sr[i + 2 * q + 1]));
+          mx = (float)max(max(m4[0], m4[1]), max(m4[2], m4[3])) * sc;  // a member row has a real key
+        } else {
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
+          }
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 64; i += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
+          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sc;
         }
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (!((vm >> i) & 1ull)) sr[i] = __float_as_uint(-INFINITY);
-        }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int i = 0; i < 64; i += 8)
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
-        mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sc;
       }
       if (!i8) {  // 4-bit units share one S buffer: release it at once
         tc_fence_before();
@@ -817,11 +821,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (member) {
         const uint64_t scx2 = f2pack(sc, sc), negr = f2pack(-r_use, -r_use);
         uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-        // p = exp2(s*sc - r) in place of the scores
+        // p = exp2(s*sc - r) in place of the scores (INT8: the exact s32 ->
+        // fp32 conversion first, through the mantissa of 1.5*2^23, |S| < 2^22)
+        const uint64_t kx2 = f2pack(-kI8BiasF, -kI8BiasF);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
+          uint64_t sp = f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+          if (i8) sp = f2add(f2pack(__uint_as_float(sr[2 * i] + kI8Bias), __uint_as_float(sr[2 * i + 1] + kI8Bias)), kx2);
           float x0, x1;
-          f2unpack(f2fma(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), scx2, negr), x0, x1);
+          f2unpack(f2fma(sp, scx2, negr), x0, x1);
           float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
           if (!full) {  // padding keys contribute nothing, whatever the block scale (sc may be 0)
             if (!((vm >> (2 * i)) & 1ull)) p0 = 0.f;
