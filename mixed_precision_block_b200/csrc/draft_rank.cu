@@ -7,7 +7,7 @@
 // ties by ascending pair index) hands out 16-bit, then INT8, then NVFP4, and
 // the rest of the pairs are skipped.
 //
-// draft_logits   fp32 SIMT GEMM tiles (64x64, both maps at once) → raw logits
+// draft_logits   fp32 SIMT GEMM tiles (128x128, 8x8 per thread) → raw logits of both maps
 // draft_mix      one CTA per query region: row softmaxes, the mix, and the
 //                first radix-select histogram of the ranking keys
 // rank_*         MSD radix select, 8 bits per pass, of the three cut keys on
@@ -23,10 +23,12 @@
 namespace da2 {
 namespace {
 
-constexpr int kTile = 64;
-constexpr int kKc = 32;
 
-__global__ void __launch_bounds__(256) draft_logits_kernel(Geom g, const float* __restrict__ qa,
+// Logit tiles of 128 x 128 region pairs, both maps one after the other: 256
+// threads, each 8 x 8 outputs (rows ty*4.. and 64+ty*4.., columns tx*4.. and
+// 64+tx*4..), so a k step is four 16-byte shared loads for 64 FMAs.
+constexpr int kLT = 128, kLK = 16;
+__global__ void __launch_bounds__(256, 2) draft_logits_kernel(Geom g, const float* __restrict__ qa,
                                                            const float* __restrict__ ka,
                                                            const float* __restrict__ qm,
                                                            const float* __restrict__ km,
@@ -34,52 +36,89 @@ __global__ void __launch_bounds__(256) draft_logits_kernel(Geom g, const float* 
                                                            float* __restrict__ lb) {
   const int D = g.d, nb = g.nb;
   const int bh = blockIdx.z;
-  const int r0 = blockIdx.y * kTile, c0 = blockIdx.x * kTile;
+  const int r0 = blockIdx.y * kLT, c0 = blockIdx.x * kLT;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  __shared__ __align__(16) float sA[2][kKc][kTile + 4];  // [map][k][row]
-  __shared__ float sB[2][kKc][kTile + 1];                // [map][k][col]
+  __shared__ __align__(16) float sA[2][kLK][kLT];  // [buffer][k][row]
+  __shared__ __align__(16) float sB[2][kLK][kLT];  // [buffer][k][col]
   const size_t base = (size_t)bh * nb * D;
-  float acc[2][4][4] = {};
-  for (int k0 = 0; k0 < D; k0 += kKc) {
-    // 2 maps x 64 rows x 32 k for each of A and B: 4096 values each, 16 per thread
-    for (int e = tid; e < kTile * kKc; e += 256) {
-      const int r = e / kKc, kk = e % kKc;
-      const int gr = r0 + r, gc = c0 + r;
-      sA[0][kk][r] = gr < nb ? qa[base + (size_t)gr * D + k0 + kk] : 0.f;
-      sA[1][kk][r] = gr < nb ? qm[base + (size_t)gr * D + k0 + kk] : 0.f;
-      sB[0][kk][r] = gc < nb ? ka[base + (size_t)gc * D + k0 + kk] : 0.f;
-      sB[1][kk][r] = gc < nb ? km[base + (size_t)gc * D + k0 + kk] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kKc; ++kk) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const float4 a4 = *reinterpret_cast<const float4*>(&sA[m][kk][ty * 4]);
-        const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-        float b[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) b[j] = sB[m][kk][tx + 16 * j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[m][i][j] = fmaf(a[i], b[j], acc[m][i][j]);
-      }
-    }
-    __syncthreads();
-  }
   const float sc = 1.0f / sqrtf((float)D);
+  const bool vec_out = (nb & 3) == 0;
+  const int nk = D / kLK;
+#pragma unroll 1
+  for (int m = 0; m < 2; ++m) {
+    const float* __restrict__ A = m ? qm : qa;
+    const float* __restrict__ B = m ? km : ka;
+    float* __restrict__ O = m ? lb : la;
+    float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty * 4 + i;
-    if (r >= nb) continue;
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx + 16 * j;
-      if (c < nb) {
-        const size_t o = ((size_t)bh * nb + r) * nb + c;
-        la[o] = acc[0][i][j] * sc;
-        lb[o] = acc[1][i][j] * sc;
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    // 128 rows x 16 k of A and of B per chunk: 512 float4 each, two per
+    // thread, fetched into registers one chunk ahead of the shared tiles
+    float4 av[2], bv[2];
+    auto fetch = [&](int k0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int e = tid + 256 * t, r = e >> 2, kq = e & 3;
+        const int gr = r0 + r, gc = c0 + r;
+        av[t] = gr < nb ? *reinterpret_cast<const float4*>(A + base + (size_t)gr * D + k0 + 4 * kq)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        bv[t] = gc < nb ? *reinterpret_cast<const float4*>(B + base + (size_t)gc * D + k0 + 4 * kq)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int e = tid + 256 * t, r = e >> 2, kq = e & 3;
+        sA[buf][4 * kq][r] = av[t].x; sA[buf][4 * kq + 1][r] = av[t].y;
+        sA[buf][4 * kq + 2][r] = av[t].z; sA[buf][4 * kq + 3][r] = av[t].w;
+        sB[buf][4 * kq][r] = bv[t].x; sB[buf][4 * kq + 1][r] = bv[t].y;
+        sB[buf][4 * kq + 2][r] = bv[t].z; sB[buf][4 * kq + 3][r] = bv[t].w;
+      }
+    };
+    fetch(0);
+    stash(0);
+    __syncthreads();
+#pragma unroll 1
+    for (int kc = 0; kc < nk; ++kc) {
+      const int buf = kc & 1;
+      if (kc + 1 < nk) fetch((kc + 1) * kLK);
+#pragma unroll
+      for (int kk = 0; kk < kLK; ++kk) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&sA[buf][kk][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&sA[buf][kk][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&sB[buf][kk][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&sB[buf][kk][64 + tx * 4]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      if (kc + 1 < nk) stash(buf ^ 1);
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+      if (r >= nb) continue;
+      float* __restrict__ orow = O + ((size_t)bh * nb + r) * nb;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + 64 * h + tx * 4;
+        const float v0 = acc[i][4 * h] * sc, v1 = acc[i][4 * h + 1] * sc;
+        const float v2 = acc[i][4 * h + 2] * sc, v3 = acc[i][4 * h + 3] * sc;
+        if (vec_out && c + 3 < nb) {
+          *reinterpret_cast<float4*>(orow + c) = make_float4(v0, v1, v2, v3);
+        } else {
+          if (c < nb) orow[c] = v0;
+          if (c + 1 < nb) orow[c + 1] = v1;
+          if (c + 2 < nb) orow[c + 2] = v2;
+          if (c + 3 < nb) orow[c + 3] = v3;
+        }
       }
     }
   }
@@ -314,7 +353,7 @@ __global__ void __launch_bounds__(256) rank_assign_kernel(Geom g, const float* _
 cudaError_t launch_draft(const Geom& g, const Layout& L, void* ws, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(at<char>(ws, L, R_HIST), 0, L.size[R_HIST], st);
   if (e != cudaSuccess) return e;
-  const int t = (g.nb + kTile - 1) / kTile;
+  const int t = (g.nb + kLT - 1) / kLT;
   draft_logits_kernel<<<dim3(t, t, g.BH), 256, 0, st>>>(
       g, at<float>(ws, L, R_Q_AVG), at<float>(ws, L, R_K_AVG), at<float>(ws, L, R_Q_MAX),
       at<float>(ws, L, R_K_MAX), at<float>(ws, L, R_SCORES), at<float>(ws, L, R_LOGB));
