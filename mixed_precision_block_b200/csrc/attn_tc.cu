@@ -1004,43 +1004,95 @@ namespace {
 // Merged key lists of query-block pairs (2p, 2p+1): per phase (16, 8, 4) the
 // ascending key blocks either member keeps in that phase, with member flags and
 // a flag for key blocks without padding.
+// Per phase, the key blocks either query block of the pair keeps, in the
+// order the attention kernel takes them two at a time: ascending, except that
+// when the pair has no 16-bit block (so nothing has set the low-bit phases'
+// P reference) a low-bit phase takes first the blocks both query blocks keep,
+// the likeliest to hold a row's largest scores, so that the reference rises
+// early and seldom later; each group ascending.  The two map rows are staged
+// in shared memory once for all passes.
 __global__ void __launch_bounds__(256) pair_lists_kernel(Geom g, const uint8_t* __restrict__ map,
                                                          uint32_t* __restrict__ plist, int* __restrict__ pcnt,
                                                          int npairs) {
   const int pair = blockIdx.x, bh = blockIdx.y, nb = g.nb;
   const int qa = 2 * pair, qb = (2 * pair + 1 < nb) ? 2 * pair + 1 : -1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint8_t* ra = map + ((size_t)bh * nb + qa) * nb;
-  const uint8_t* rb = qb >= 0 ? map + ((size_t)bh * nb + qb) * nb : nullptr;
+  extern __shared__ uint8_t rows_sm[];  // [2][nb]
+  {
+    const uint8_t* ga = map + ((size_t)bh * nb + qa) * nb;
+    const uint8_t* gb = qb >= 0 ? map + ((size_t)bh * nb + qb) * nb : nullptr;
+    for (int i = threadIdx.x; i < nb; i += 256) {
+      rows_sm[i] = ga[i];
+      rows_sm[nb + i] = gb ? gb[i] : (uint8_t)0;
+    }
+    __syncthreads();
+  }
+  const uint8_t* ra = rows_sm;
+  const uint8_t* rb = qb >= 0 ? rows_sm + nb : nullptr;
   uint32_t* out = plist + ((size_t)bh * npairs + pair) * (2 * nb);
-  __shared__ int wtot[8];
+  __shared__ int wtot[3][8];
+  __shared__ int tot[3];
   int run = 0;
   int counts[3];
   const int phase_bits[3] = {16, 8, 4};
   for (int ph = 0; ph < 3; ++ph) {
     const int start = run;
+    // class of a key block: 0 both keep it, 1 only one of them does
+    auto cls = [&](int kb) -> int {
+      if (kb >= nb) return -1;
+      const bool a = ra[kb] == phase_bits[ph], b = rb && rb[kb] == phase_bits[ph];
+      return (a && b && ph > 0 && counts[0] == 0) ? 0 : ((a || b) ? 1 : -1);
+    };
+    // pass 1 (only when some block can come first): the class sizes
+    int n[3] = {0, 0, 0};
+    const bool two_groups = ph > 0 && counts[0] == 0;
+    for (int base = 0; two_groups && base < nb; base += 256) {
+      const int c = cls(base + threadIdx.x);
+#pragma unroll
+      for (int k = 0; k < 3; ++k) n[k] += __popc(__ballot_sync(0xffffffffu, c == k));
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < 3; ++k) wtot[k][warp] = n[k];
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+      int t = 0;
+      for (int w = 0; w < 8; ++w) t += wtot[threadIdx.x][w];
+      tot[threadIdx.x] = t;
+    }
+    __syncthreads();
+    const int nc = tot[0];  // the first group's size (0 for one ascending group)
+    __syncthreads();
+    // pass 2: each entry at its place
+    int seen[3] = {0, 0, 0};  // entries of each class before this chunk
     for (int base = 0; base < nb; base += 256) {
       const int kb = base + threadIdx.x;
-      bool a = false, b = false;
-      if (kb < nb) {
-        a = ra[kb] == phase_bits[ph];
-        b = rb && rb[kb] == phase_bits[ph];
+      const int c = cls(kb);
+      unsigned bal[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) bal[k] = __ballot_sync(0xffffffffu, c == k);
+      if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) wtot[k][warp] = __popc(bal[k]);
       }
-      const unsigned bal = __ballot_sync(0xffffffffu, a || b);
-      if (lane == 0) wtot[warp] = __popc(bal);
       __syncthreads();
-      if (a || b) {
-        int off = run;
-        for (int w = 0; w < warp; ++w) off += wtot[w];
-        off += __popc(bal & ((1u << lane) - 1u));
+      if (c >= 0) {
+        int i = seen[c] + __popc(bal[c] & ((1u << lane) - 1u));  // rank within the class
+        for (int w = 0; w < warp; ++w) i += wtot[c][w];
+        const int off = c == 0 ? i : nc + i;
         const int rx = kb % g.nrx, ry = (kb / g.nrx) % g.nry;
         const bool full = (ry + 1) * g.rh <= g.Hh && (rx + 1) * g.rw <= g.Ww;
-        out[off] = (uint32_t)kb | ((uint32_t)a << 16) | ((uint32_t)b << 17) | ((uint32_t)ph << 18) |
-                   ((uint32_t)full << 20);
+        const bool a = ra[kb] == phase_bits[ph], b = rb && rb[kb] == phase_bits[ph];
+        out[start + off] = (uint32_t)kb | ((uint32_t)a << 16) | ((uint32_t)b << 17) | ((uint32_t)ph << 18) |
+                           ((uint32_t)full << 20);
       }
-      for (int w = 0; w < 8; ++w) run += wtot[w];
+#pragma unroll
+      for (int k = 0; k < 3; ++k)
+        for (int w = 0; w < 8; ++w) seen[k] += wtot[k][w];
       __syncthreads();
     }
+    run = start + seen[0] + seen[1];
     counts[ph] = run - start;
   }
   if (threadIdx.x == 0)
@@ -1141,8 +1193,14 @@ cudaError_t launch_dense_tc(int B, int H, int N, const void* q, const void* k, c
 
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st) {
   const int npairs = (g.nb + 1) / 2;
-  pair_lists_kernel<<<dim3(npairs, g.BH), 256, 0, st>>>(g, at<uint8_t>(ws, L, R_MAP), at<uint32_t>(ws, L, R_PLIST),
-                                                       at<int>(ws, L, R_PCNT), npairs);
+  const size_t smem = (2 * (size_t)g.nb + 15) & ~(size_t)15;  // the pair's two map rows
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(pair_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  pair_lists_kernel<<<dim3(npairs, g.BH), 256, smem, st>>>(g, at<uint8_t>(ws, L, R_MAP), at<uint32_t>(ws, L, R_PLIST),
+                                                          at<int>(ws, L, R_PCNT), npairs);
   return cudaGetLastError();
 }
 

@@ -19,10 +19,13 @@ Readings adopted (the pages leave these open):
   product of the INT8 codes times both block scales; 4-bit phase from the
   dequantised NVFP4 values; all times 1/sqrt(d).  Padding keys score -inf.
 * key blocks are taken two at a time ("units"), in the order a kernel that
-  pairs neighbouring query blocks (2p, 2p+1) walks them: per phase, the union
-  of the two query blocks' key-block lists in ascending order, cut into
-  consecutive pairs.  A unit's blocks that this query block does not retain
-  contribute nothing to its rows.
+  pairs neighbouring query blocks (2p, 2p+1) walks them: per low-bit phase,
+  the key blocks either query block retains, ascending; when neither query
+  block of the pair retains a 16-bit block (nothing has set the reference),
+  first those both retain, then the rest, each group ascending.  The list is
+  cut into consecutive pairs.  A unit's blocks that this query block does not
+  retain contribute nothing to its rows.  (The 16-bit phase's result does not
+  depend on the order.)
 * P in the 8-bit and 4-bit phases is quantised relative to a running power of
   two 2^r per row (r an integer, log2 units).  The phases share the softmax
   statistics, so a low-bit phase starts from r = ceil(x_run), x_run the row's
@@ -86,14 +89,19 @@ class _State:
         self.m = m_new
 
 
-def phase_units(prec_row, partner_row, bit):
-    """The units of one phase: the key blocks that this query block or its
-    partner (the other block of its pair) assign to ``bit``, ascending, cut into
-    consecutive pairs (the last may hold one block)."""
-    sel = prec_row == bit
-    if partner_row is not None:
-        sel = sel | (partner_row == bit)
-    kbs = np.nonzero(sel)[0]
+def phase_units(even_row, odd_row, bit):
+    """The units of one low-bit phase of the query-block pair (2p, 2p+1),
+    whose precision rows are ``even_row`` and ``odd_row`` (None if 2p+1 does
+    not exist): the key blocks either assigns to ``bit``, ascending; if
+    neither row holds a 16-bit block, those both assign first, then the rest,
+    each group ascending.  Cut into consecutive pairs (the last may hold one)."""
+    a = even_row == bit
+    b = odd_row == bit if odd_row is not None else np.zeros_like(a)
+    no16 = not np.any(even_row == BIT16) and (odd_row is None or not np.any(odd_row == BIT16))
+    if no16:
+        kbs = np.concatenate([np.nonzero(a & b)[0], np.nonzero(a ^ b)[0]]).astype(np.int64)
+    else:
+        kbs = np.nonzero(a | b)[0].astype(np.int64)
     return [kbs[i:i + 2] for i in range(0, len(kbs), 2)]
 
 
@@ -151,7 +159,9 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None, tr
     ``prep``: dict from ``prep.prepare_head``; ``prec_row``: uint8 [nb] precision
     of each key block for this query block (16, 8, 4, 0); ``partner_row``: the
     same for the other query block of its pair (qb ^ 1), None if there is none.
-    The partner only decides how the low-bit phases group key blocks into units.
+    The partner only decides how the low-bit phases group key blocks into units
+    (``qb`` even: this block is the pair's even one; a missing partner leaves
+    this block's own list).
     ``trace``: a dict that receives each low-bit phase's starting reference
     (``r0_8``, ``r0_4``, per row)."""
     S = prep["q_blocks"].shape[1]
@@ -189,7 +199,8 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None, tr
     ph = _LowBitPhase(S, d, np.ceil(x_run))
     if trace is not None:
         trace["r0_8"] = ph.r.copy()
-    for unit in phase_units(prec_row, partner_row, BIT8):
+    even, odd = (prec_row, partner_row) if (qb % 2 == 0 or partner_row is None) else (partner_row, prec_row)
+    for unit in phase_units(even, odd, BIT8):
         xs = []
         for kb in unit:
             s_int = qi @ prep["k_i8"][kb].astype(np.float64).T  # exact integers
@@ -207,7 +218,7 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None, tr
     ph = _LowBitPhase(S, d, np.ceil(x_run))
     if trace is not None:
         trace["r0_4"] = ph.r.copy()
-    for unit in phase_units(prec_row, partner_row, BIT4):
+    for unit in phase_units(even, odd, BIT4):
         xs = []
         for kb in unit:
             kd = F.nvfp4_dequantize(prep["k_f4"][kb], prep["k_sf4"][kb])

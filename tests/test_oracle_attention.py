@@ -151,13 +151,42 @@ def test_scatter_restores_token_order():
     np.testing.assert_array_equal(attention.scatter(blocks, tab, p.N), x)
 
 
-def test_phase_units_union_of_the_pair_in_pairs():
-    # this query block keeps 8-bit blocks 0, 2, 3; its partner 1, 3, 4
-    row = np.array([8, 0, 8, 8, 0], dtype=np.uint8)
-    partner = np.array([0, 8, 0, 8, 8], dtype=np.uint8)
-    units = [list(u) for u in attention.phase_units(row, partner, 8)]
-    assert units == [[0, 1], [2, 3], [4]]
-    assert [list(u) for u in attention.phase_units(row, None, 8)] == [[0, 2], [3]]
+def test_phase_units_order_of_the_pair():
+    # the even block keeps 8-bit blocks 0, 2, 3, 5, 6; the odd one 1, 3, 4.
+    # No 16-bit block in the pair: 3 (kept by both) first, then 0 1 2 4 5 6,
+    # cut in pairs, from either side
+    row = np.array([8, 0, 8, 8, 0, 8, 8, 0], dtype=np.uint8)
+    partner = np.array([0, 8, 0, 8, 8, 0, 0, 0], dtype=np.uint8)
+    want = [[3, 0], [1, 2], [4, 5], [6]]
+    assert [list(u) for u in attention.phase_units(row, partner, 8)] == want
+    assert [list(u) for u in attention.phase_units(partner, row, 8)] == want
+    # a 16-bit block anywhere in the pair (block 7 of the odd row): the union ascending
+    p16 = partner.copy()
+    p16[7] = 16
+    assert [list(u) for u in attention.phase_units(row, p16, 8)] == [[0, 1], [2, 3], [4, 5], [6]]
+    # a block alone: its own list ascending; other precisions are not in the phase
+    assert [list(u) for u in attention.phase_units(row, None, 8)] == [[0, 2], [3, 5], [6]]
+    assert attention.phase_units(row, partner, 4) == []
+
+
+def test_unit_order_covers_every_retained_block():
+    # Q = 0 makes every score 0, so the order cannot change the result, but
+    # the unit order must still cover every retained block exactly once: the
+    # closed form of the 8-bit phase (code 255 everywhere: the mean of the
+    # INT8-dequantised V of the retained blocks)
+    p, q, k, v = _inputs(Hh=12, Ww=10, budget=(40, 0, 60, 0))
+    q = np.zeros_like(q)
+    r = pipeline.run_head(p, q, k, v, mode="math")
+    pr = r["prep"]
+    vb = pr["v_i8"].astype(np.float64) * pr["v_s8"][None, :, None]  # [nb, d, S]
+    for qb in range(p.nb):
+        keep = np.nonzero(r["map"][qb] == 8)[0]
+        if len(keep) == 0:
+            continue
+        vt = np.concatenate([vb[b][:, pr["valid"][b]] for b in keep], axis=1)
+        rows = pr["valid"][qb]
+        got = attention.qblock_attention(pr, qb, r["map"][qb], p.d, "math", attention.partner_of(r["map"], qb))
+        np.testing.assert_allclose(got[rows], np.broadcast_to(vt.mean(1), (rows.sum(), p.d)), rtol=1e-12)
 
 
 def test_low_bit_reference_raise_by_hand():
