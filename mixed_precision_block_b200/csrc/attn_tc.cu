@@ -31,14 +31,17 @@
 //           for the P·V of the one before unless O must be rescaled.
 //   Low-bit phases accumulate P·V in TMEM at column 384 (INT8: s32 X8; 4-bit:
 //   fp32 O4) against a power-of-two reference 2^r per row, shared by the two
-//   warps of the row and raised to ceil(unit max) whenever a unit's max
-//   exceeds it; P is quantised relative to 2^r.  Before a raise (INT8 also
+//   warps of the row, starting from ceil of the row's running max over all
+//   earlier units (the shared softmax statistics) and raised to ceil(unit
+//   max) whenever a unit's max exceeds it; P is quantised relative to 2^r.  Before a raise (INT8 also
 //   every 256 units, ahead of s32 overflow) and at the end of the phase the
 //   accumulator is folded into O with the phase's channel scale (sv/255 or
 //   g/2688) and cleared.
-//   8-bit   S = Q8·[K8_a; K8_b]^T (kind::i8, s32 read back exactly through the
-//           mantissa of 1.5·2^23); codes rint(255 p) as u8 replace the scores
-//           in TMEM; X8 += P8·V8 (kind::i8 u8×s8, A from TMEM).
+//   8-bit   S = Q8·[K8_a; K8_b]^T (kind::i8, s32); the row max is taken on
+//           the integers, the exact fp32 scores (through the mantissa of
+//           1.5·2^23) only after the max exchange; codes rint(255 p) as u8
+//           replace the scores in TMEM; X8 += P8·V8 (kind::i8 u8×s8, A from
+//           TMEM).
 //   4-bit   S_h = Q4·K4_h^T (kind::mxf4nvf4, block16 e4m3 scales copied into
 //           TMEM with tcgen05.cp from the scale atoms prep wrote); 2688 p
 //           quantised to NVFP4 per 16 keys in registers, codes and scale atom
