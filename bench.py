@@ -61,6 +61,37 @@ XU_LANES_PER_CLK_SM = 16
 SMS = 148
 
 
+def attention_roofline(wl, info, attn_ms, pk, pk_kind, mhz):
+    """Roofline of the attention kernel against the larger of two floors: the
+    tensor floor (each phase's executed MMA FLOPs at its format's peak, bf16
+    the measured sustained figure, INT8 x2, NVFP4 x4) and the softmax's XU
+    floor (XU_PER_PAIR per retained pair at XU_LANES_PER_CLK_SM lanes per
+    clock per SM at the sampled SM clock)."""
+    sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    pf = phase_flops(wl, info)
+    f_tot = sum(pf.values())
+    t_roof_s = pf[16] / (sus * 1e12) + pf[8] / (2 * sus * 1e12) + pf[4] / (4 * sus * 1e12)
+    bh = wl.B * wl.H
+    xu_ops = bh * (info.n16 * XU_PER_PAIR[16] + info.n8 * XU_PER_PAIR[8] + info.n4 * XU_PER_PAIR[4])
+    xu_peak = XU_LANES_PER_CLK_SM * SMS * mhz * 1e6  # ops/s
+    floors_ms = {"tensor": t_roof_s * 1e3, "xu": xu_ops / xu_peak * 1e3}
+    if floors_ms["xu"] > floors_ms["tensor"]:
+        roof = {"bound": "alu", "achieved": xu_ops / (attn_ms * 1e-3) / 1e9, "peak": xu_peak / 1e9,
+                "unit": "Gop/s", "frac": floors_ms["xu"] / attn_ms,
+                "peak_note": f"XU pipe (ex2 + F2FP conversions), {XU_LANES_PER_CLK_SM} lanes/clk/SM x {SMS} SMs "
+                             f"at {mhz:.0f} MHz; tensor floor {floors_ms['tensor']:.2f} ms is lower"}
+    else:
+        achieved = f_tot / (attn_ms * 1e-3) / 1e12
+        peak_blend = f_tot / t_roof_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_blend, "unit": "TFLOP/s",
+                "frac": achieved / peak_blend,
+                "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
+                             f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
+                             f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"}
+    roof["floors_ms"] = floors_ms
+    return roof
+
+
 def max_over_ranks(x, device, world):
     """The largest of the ranks' values; every rank takes the same collective."""
     if world <= 1:
@@ -346,37 +377,12 @@ def run_ours(args, wl):
                "call": f"da2_forward_host on pinned host tensors, chunks of {args.e2e_chunk} (batch, head) slices"}
         del hq, hk, hv, hout, hbuf
 
-    pk, pk_kind = peaks()
-    sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    pf = phase_flops(wl, info)
-    f_tot = sum(pf.values())
-    t_roof_s = pf[16] / (sus * 1e12) + pf[8] / (2 * sus * 1e12) + pf[4] / (4 * sus * 1e12)
-    attn_ms = stage[2]
-    achieved = f_tot / (attn_ms * 1e-3) / 1e12
-    peak_blend = f_tot / t_roof_s / 1e12
     kname, ksrc = roofline_kernel(wl)
     traffic = traffic_record(kname, os.path.join(ROOT, "mixed_precision_block_b200", "csrc", ksrc), wl.name)
     clocks = clk.summary()
-    # the softmax's XU floor beside the tensor floor; the larger one bounds the kernel
-    bh = wl.B * wl.H
-    xu_ops = bh * (info.n16 * XU_PER_PAIR[16] + info.n8 * XU_PER_PAIR[8] + info.n4 * XU_PER_PAIR[4])
-    mhz = (clocks or {}).get("sm_mhz") or 1965.0
-    xu_peak = XU_LANES_PER_CLK_SM * SMS * mhz * 1e6  # ops/s
-    floors_ms = {"tensor": t_roof_s * 1e3, "xu": xu_ops / xu_peak * 1e3}
-    if floors_ms["xu"] > floors_ms["tensor"]:
-        roof = {"bound": "alu", "kernel": kname, "achieved": xu_ops / (attn_ms * 1e-3) / 1e9,
-                "peak": xu_peak / 1e9, "unit": "Gop/s", "frac": floors_ms["xu"] / attn_ms,
-                "traffic": traffic,
-                "peak_note": f"XU pipe (ex2 + F2FP conversions), {XU_LANES_PER_CLK_SM} lanes/clk/SM x {SMS} SMs "
-                             f"at {mhz:.0f} MHz; tensor floor {floors_ms['tensor']:.2f} ms is lower"}
-    else:
-        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved,
-                "peak": peak_blend, "unit": "TFLOP/s", "frac": achieved / peak_blend,
-                "traffic": traffic,
-                "peak_note": f"phase-weighted: bf16 {sus:.0f} (sustained, {pk_kind}), "
-                             f"int8 x2, nvfp4 x4; executed FLOPs 16/8/4 = "
-                             f"{pf[16] / 1e12:.2f}/{pf[8] / 1e12:.2f}/{pf[4] / 1e12:.2f} T"}
-    roof["floors_ms"] = floors_ms
+    pk, pk_kind = peaks()
+    roof = attention_roofline(wl, info, stage[2], pk, pk_kind, (clocks or {}).get("sm_mhz") or 1965.0)
+    roof.update(kernel=kname, traffic=traffic)
 
     if rank == 0:
         cpu = None

@@ -65,3 +65,25 @@ def test_reference_arm_is_rank_zero_only(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(None, WORKLOADS["video"])  # returns before touching its arguments
     assert buf.getvalue() == ""
+
+
+def test_roofline_takes_the_larger_floor():
+    sys.path.insert(0, ROOT)
+    import bench
+    from types import SimpleNamespace
+    from mixed_precision_block_b200.synth import WORKLOADS
+    pk = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    wl = WORKLOADS["video"]  # 24 heads
+    # 16-bit only: tensor floor = 4*64*64*128 FLOP * n16 * 24 / 1.4e15; XU = 6144 ops * n16 * 24 / (16*148*1965e6)
+    info = SimpleNamespace(n16=1000, n8=0, n4=0)
+    r = bench.attention_roofline(wl, info, 1.0, pk, "measured", 1965.0)
+    t_tensor = 4 * 64 * 64 * 128 * 1000 * 24 / 1.4e15 * 1e3
+    t_xu = 6144 * 1000 * 24 / (16 * 148 * 1965e6) * 1e3
+    assert abs(r["floors_ms"]["tensor"] - t_tensor) < 1e-12 and abs(r["floors_ms"]["xu"] - t_xu) < 1e-12
+    assert r["bound"] == ("tensor" if t_tensor >= t_xu else "alu")
+    assert abs(r["frac"] - max(t_tensor, t_xu) / 1.0) < 1e-12  # achieved/peak = floor/time
+    # 4-bit only: the tensor floor is a quarter, the XU floor larger: bound by the XU pipe
+    info = SimpleNamespace(n16=0, n8=0, n4=1000)
+    r = bench.attention_roofline(wl, info, 1.0, pk, "measured", 1965.0)
+    assert r["bound"] == "alu" and r["unit"] == "Gop/s"
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
