@@ -6,48 +6,45 @@ the softmax statistics (running max and sum) and one output accumulator, and
 quantisation scales are folded in at the phase boundaries, so no partial
 outputs are written back and merged.  Skipped pairs contribute nothing.
 
-This module follows that structure literally, per query block, in fp64:
-phase 16, then phase 8, then phase 4, one online-softmax state (m, l, O)
-carried across all of them; each low-bit phase accumulates in its own
-accumulator against a power-of-two reference that starts from the running
-maximum of the phases before it, and is folded into that state, with its
-channel scales, at the phase boundary.
+This module follows that structure per query block, in fp64: phase 16, then
+phase 8, then phase 4.  Every retained key block contributes a partial
+(reference m_blk, sum l_blk, numerator x_blk) that is merged into one
+online-softmax state (m, l, O); a low-bit phase gathers its blocks' numerators
+in the units of its quantised operands and applies the V channel scale once,
+at the phase boundary.  The result depends only on the query block's own
+precision row: no block's contribution depends on another block's, so the
+order in which blocks are visited (and any grouping a kernel uses) does not
+change it beyond rounding.
 
 Readings adopted (the pages leave these open):
 
-* scores: 16-bit phase from the bf16 values; 8-bit phase from the exact integer
-  product of the INT8 codes times both block scales; 4-bit phase from the
-  dequantised NVFP4 values; all times 1/sqrt(d).  Padding keys score -inf.
-* key blocks are taken two at a time ("units"), in the order a kernel that
-  pairs neighbouring query blocks (2p, 2p+1) walks them: per low-bit phase,
-  the key blocks either query block retains, ascending; when neither query
-  block of the pair retains a 16-bit block (nothing has set the reference),
-  first those both retain, then the rest, each group ascending.  The list is
-  cut into consecutive pairs.  A unit's blocks that this query block does not
-  retain contribute nothing to its rows.  (The 16-bit phase's result does not
-  depend on the order.)
-* P in the 8-bit and 4-bit phases is quantised relative to a running power of
-  two 2^r per row (r an integer, log2 units).  The phases share the softmax
-  statistics, so a low-bit phase starts from r = ceil(x_run), x_run the row's
-  running maximum of s·log2 e over every unit of the phases before it (-inf
-  if there was none).  Before a unit, if the unit's row maximum x_max (over
-  its retained keys) exceeds r, r becomes ceil(x_max), and what the phase
-  accumulated so far is scaled by 2^(r_old - r).  So p = 2^(x - r) is in
-  (0, 1]:
-  8-bit code = round(255 p) as an unsigned byte (scale 1/255);
-  4-bit = NVFP4, over 16 consecutive keys of the row, of 2688 p (2688 = 6·448
-  puts the largest p at the top of the e2m1 x e4m3 range), dequantised and
-  divided by 2688 again.  Each phase accumulates its P·V in its own
-  accumulator; the phases' results meet, with the channel scales, at the end.
-* the softmax denominator l sums the unquantised exp(s - m) over every retained
-  real key of every phase.
+* scores: 16-bit phase from the bf16 values; 8-bit phase from the exact
+  integer product of the INT8 codes times both block scales; 4-bit phase from
+  the dequantised NVFP4 values; all times 1/sqrt(d).  Padding keys score -inf.
+* low-bit P is quantised per (query row, key block), relative to that block's
+  own row maximum, so that every retained block keeps the full resolution of
+  its format whatever its rank in the row (the reading note, Method overview
+  bullet 3: low-bit precision recovers the mid-importance interactions):
+  - 8-bit: p = exp(s - m_blk) in (0, 1], m_blk the block's row maximum;
+    code = round(255 p) as an unsigned byte; the block's weights are code/255
+    times exp(m_blk - m);
+  - 4-bit: with x = s log2 e, the reference is r_blk = ceil(max x), the
+    block's row maximum rounded up to a power of two; p = 2^(x - r_blk) in
+    (0, 1] is quantised as NVFP4 of 2688 p over 16 consecutive keys of the
+    row (2688 = 6 x 448 puts the largest possible p at the top of the
+    e2m1 x e4m3 range), dequantised and divided by 2688; the block's weights
+    are that times 2^r_blk.  A power of two passes through the e4m3 scale
+    exactly, so the same codes come out against any larger power-of-two
+    reference while the microblock scale stays normal (>= 2^-6).
+* the softmax denominator sums, per phase, the weights the numerator uses:
+  unquantised p in the 16-bit phase, the quantised weights above in the
+  low-bit phases (so each low-bit block enters numerator and denominator with
+  the same weights and the output stays a weighted mean of V).
 * 16-bit phase, ``emulate`` mode: P is rounded to bf16 relative to a power of
-  two, 2^r with r = ceil(m_run * log2 e) and m_run the running maximum over the
-  16-bit blocks seen so far (ascending key blocks).  Because bf16 rounding
-  commutes with scaling by powers of two, the rounded P is then the same for
-  any integer-exponent reference a kernel keeps, however lazily it raises it
-  (parity unpinned beyond that: the GPU's exponential).  ``math`` mode keeps P
-  exact.
+  two, 2^ceil(max x) over the block; bf16 rounding commutes with scaling by
+  powers of two, so this is the rounding against any integer-exponent
+  reference a kernel keeps (parity unpinned beyond that: the GPU's
+  exponential).  ``math`` mode keeps P exact.
 * ``emulate`` mode rounds the output to bf16; a query block with no retained
   key block outputs zeros.
 """
@@ -73,13 +70,16 @@ def bf16_round(x):
 
 
 class _State:
+    """Online-softmax state shared by every phase: per row a reference m, the
+    sum l and the numerator O, both relative to exp(m)."""
+
     def __init__(self, rows, d):
         self.m = np.full(rows, -np.inf)
         self.l = np.zeros(rows)
         self.o = np.zeros((rows, d))
 
     def merge(self, m_blk, l_blk, x_blk):
-        """Merge a block whose P was taken relative to m_blk (per row)."""
+        """Merge a partial whose weights were taken relative to exp(m_blk)."""
         m_new = np.maximum(self.m, m_blk)
         ok = np.isfinite(m_new)
         a_old = np.where(ok & np.isfinite(self.m), np.exp(self.m - np.where(ok, m_new, 0)), 0.0)
@@ -87,60 +87,6 @@ class _State:
         self.l = self.l * a_old + l_blk * a_blk
         self.o = self.o * a_old[:, None] + x_blk * a_blk[:, None]
         self.m = m_new
-
-
-def phase_units(even_row, odd_row, bit):
-    """The units of one low-bit phase of the query-block pair (2p, 2p+1),
-    whose precision rows are ``even_row`` and ``odd_row`` (None if 2p+1 does
-    not exist): the key blocks either assigns to ``bit``, ascending; if
-    neither row holds a 16-bit block, those both assign first, then the rest,
-    each group ascending.  Cut into consecutive pairs (the last may hold one)."""
-    a = even_row == bit
-    b = odd_row == bit if odd_row is not None else np.zeros_like(a)
-    no16 = not np.any(even_row == BIT16) and (odd_row is None or not np.any(odd_row == BIT16))
-    if no16:
-        kbs = np.concatenate([np.nonzero(a & b)[0], np.nonzero(a ^ b)[0]]).astype(np.int64)
-    else:
-        kbs = np.nonzero(a | b)[0].astype(np.int64)
-    return [kbs[i:i + 2] for i in range(0, len(kbs), 2)]
-
-
-class _LowBitPhase:
-    """A low-bit phase's P·V accumulator and sum against a running power of two
-    2^r per row (r an integer, log2 units; -inf before the first score)."""
-
-    def __init__(self, rows, d, r0=None):
-        self.r = np.full(rows, -np.inf) if r0 is None else np.array(r0, dtype=np.float64)
-        self.l = np.zeros(rows)
-        self.acc = np.zeros((rows, d))
-
-    def enter(self, xs):
-        """Take a unit whose blocks have log2-unit scores ``xs`` ([rows, keys]
-        each, -inf where not retained): raise r to ceil of the unit's row max
-        where that max exceeds r, rescale what is accumulated, add the
-        unquantised p to l and return each block's p = 2^(x - r)."""
-        x_max = np.max(np.stack([x.max(1) for x in xs]), axis=0)
-        self.x_max = x_max
-        up = np.isfinite(x_max) & (x_max > self.r)
-        r_new = np.where(up, np.ceil(np.where(up, x_max, 0.0)), self.r)
-        had = np.isfinite(self.r)
-        a = np.where(up, np.where(had, np.exp2(np.where(had, self.r, 0.0) - np.where(up, r_new, 0.0)), 0.0), 1.0)
-        self.acc *= a[:, None]
-        self.l *= a
-        self.r = r_new
-        live = np.isfinite(self.r)
-        ps = []
-        for x in xs:
-            ok = np.isfinite(x) & live[:, None]
-            p = np.where(ok, np.exp2(np.where(ok, x - np.where(live, self.r, 0.0)[:, None], 0.0)), 0.0)
-            self.l += p.sum(1)
-            ps.append(p)
-        return ps
-
-    def fold_into(self, st, chan_scale):
-        """Phase boundary: join the shared state with the phase's channel scale."""
-        m_blk = np.where(np.isfinite(self.r), self.r * LN2, -np.inf)
-        st.merge(m_blk, self.l, self.acc * chan_scale)
 
 
 def _row_max(s):
@@ -153,93 +99,86 @@ def _exp_rel(s, m):
     return np.where(ok, np.exp(np.where(ok, s - np.where(np.isfinite(m), m, 0)[:, None], 0)), 0.0)
 
 
-def qblock_attention(prep, qb, prec_row, d, mode="emulate", partner_row=None, trace=None):
+def p8_weights(s):
+    """8-bit phase weights of one key block (rows x keys, natural-log scores,
+    -inf for keys the row does not use): returns (m_blk, w) with
+    w = round(255 exp(s - m_blk)) / 255 relative to exp(m_blk)."""
+    m_blk = _row_max(s)
+    p = _exp_rel(s, m_blk)
+    return m_blk, np.rint(255.0 * p) / 255.0
+
+
+def p4_weights(x):
+    """4-bit phase weights of one key block (rows x keys, log2-unit scores,
+    -inf for unused keys): returns (r_blk, w) with r_blk = ceil(row max) and
+    w = NVFP4(2688 * 2^(x - r_blk)) / 2688 relative to 2^r_blk."""
+    xm = _row_max(x)
+    live = np.isfinite(xm)
+    r_blk = np.where(live, np.ceil(np.where(live, xm, 0.0)), -np.inf)
+    ok = np.isfinite(x) & live[:, None]
+    p = np.where(ok, np.exp2(np.where(ok, x - np.where(live, r_blk, 0.0)[:, None], 0.0)), 0.0)
+    t = F.f32(P4_RANGE * F.f32(p))
+    codes, sf = F.nvfp4_quantize(t, axis=-1, block=16)
+    return r_blk, F.nvfp4_dequantize(codes, sf) / P4_RANGE
+
+
+def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
     """Output rows [S, d] of query block ``qb`` of one head.
 
     ``prep``: dict from ``prep.prepare_head``; ``prec_row``: uint8 [nb] precision
-    of each key block for this query block (16, 8, 4, 0); ``partner_row``: the
-    same for the other query block of its pair (qb ^ 1), None if there is none.
-    The partner only decides how the low-bit phases group key blocks into units
-    (``qb`` even: this block is the pair's even one; a missing partner leaves
-    this block's own list).
-    ``trace``: a dict that receives each low-bit phase's starting reference
-    (``r0_8``, ``r0_4``, per row)."""
+    of each key block for this query block (16, 8, 4, 0)."""
     S = prep["q_blocks"].shape[1]
     valid = prep["valid"]
     inv_sqrt_d = 1.0 / np.sqrt(d)
     st = _State(S, d)
-    x_run = np.full(S, -np.inf)  # running row max of s·log2 e, every phase so far
 
-    # phase 16: bf16 operands, online softmax across blocks
+    # phase 16: bf16 operands; each block's P against its own power-of-two
+    # reference (the rounding is the same against any integer exponent)
     q = prep["q_blocks"][qb]
     for kb in np.nonzero(prec_row == BIT16)[0]:
         s = (q @ prep["k_blocks"][kb].T) * inv_sqrt_d
         s = np.where(valid[kb][None, :], s, -np.inf)
-        x_run = np.maximum(x_run, _row_max(s) * LOG2E)
-        m_new = np.maximum(st.m, _row_max(s))
+        m_blk = _row_max(s)
+        p = _exp_rel(s, m_blk)
         if mode == "emulate":
-            # P is rounded in bf16 relative to 2^ceil(m_run log2 e), then brought
-            # to the accumulator's units (exp(-m_run)) exactly
-            p_den = _exp_rel(s, m_new)
-            r = np.ceil(m_new * LOG2E)
-            shift = np.exp2(r - m_new * LOG2E)  # >= 1; exact fp64 scaling
-            p_num = bf16_round(p_den / shift[:, None]) * shift[:, None]
-            alpha = np.where(np.isfinite(st.m), np.exp(st.m - np.where(np.isfinite(m_new), m_new, 0)), 0.0)
-            st.l = st.l * alpha + p_den.sum(1)
-            st.o = st.o * alpha[:, None] + p_num @ prep["v_blocks"][kb]
-            st.m = m_new
+            live = np.isfinite(m_blk)
+            xm = np.where(live, m_blk * LOG2E, 0.0)
+            shift = np.exp2(np.ceil(xm) - xm)  # >= 1; exp(s - m_blk) = 2^(x - ceil) * shift
+            p_num = bf16_round(p / shift[:, None]) * shift[:, None]
         else:
-            m_blk = _row_max(s)
-            p = _exp_rel(s, m_blk)
-            st.merge(m_blk, p.sum(1), p @ prep["v_blocks"][kb])
+            p_num = p
+        st.merge(m_blk, p.sum(1), p_num @ prep["v_blocks"][kb])
 
-    # phase 8: INT8 Q/K codes with block scales, u8 P, INT8 V with channel scales
-    qi = prep["q_i8"][qb].astype(np.float64)
-    sq = prep["q_s8"][qb]
-    ph = _LowBitPhase(S, d, np.ceil(x_run))
-    if trace is not None:
-        trace["r0_8"] = ph.r.copy()
-    even, odd = (prec_row, partner_row) if (qb % 2 == 0 or partner_row is None) else (partner_row, prec_row)
-    for unit in phase_units(even, odd, BIT8):
-        xs = []
-        for kb in unit:
+    # phase 8: INT8 Q/K codes with block scales; u8 P against each block's own
+    # row maximum; INT8 V codes; the V channel scale applied at the boundary
+    kbs = np.nonzero(prec_row == BIT8)[0]
+    if len(kbs):
+        qi = prep["q_i8"][qb].astype(np.float64)
+        sq = prep["q_s8"][qb]
+        ph = _State(S, d)
+        for kb in kbs:
             s_int = qi @ prep["k_i8"][kb].astype(np.float64).T  # exact integers
-            s = s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d)
-            keep = valid[kb][None, :] & (prec_row[kb] == BIT8)
-            xs.append(np.where(keep, s * LOG2E, -np.inf))
-        for kb, p in zip(unit, ph.enter(xs)):
-            code = np.rint(255.0 * p)
-            ph.acc += code @ prep["v_i8"][kb].astype(np.float64).T  # exact integers
-        x_run = np.maximum(x_run, ph.x_max)
-    ph.fold_into(st, prep["v_s8"][None, :] / 255.0)
+            s = np.where(valid[kb][None, :], s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d), -np.inf)
+            m_blk, w = p8_weights(s)
+            ph.merge(m_blk, w.sum(1), w @ prep["v_i8"][kb].astype(np.float64).T)
+        st.merge(ph.m, ph.l, ph.o * prep["v_s8"][None, :])
 
-    # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks of 2688 p), NVFP4 V
-    qd = F.nvfp4_dequantize(prep["q_f4"][qb], prep["q_sf4"][qb])
-    ph = _LowBitPhase(S, d, np.ceil(x_run))
-    if trace is not None:
-        trace["r0_4"] = ph.r.copy()
-    for unit in phase_units(even, odd, BIT4):
-        xs = []
-        for kb in unit:
+    # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks of 2688 p against each
+    # block's power-of-two reference), NVFP4 V; the V channel scale g at the boundary
+    kbs = np.nonzero(prec_row == BIT4)[0]
+    if len(kbs):
+        qd = F.nvfp4_dequantize(prep["q_f4"][qb], prep["q_sf4"][qb])
+        ph = _State(S, d)
+        for kb in kbs:
             kd = F.nvfp4_dequantize(prep["k_f4"][kb], prep["k_sf4"][kb])
-            s = (qd @ kd.T) * inv_sqrt_d
-            keep = valid[kb][None, :] & (prec_row[kb] == BIT4)
-            xs.append(np.where(keep, s * LOG2E, -np.inf))
-        for kb, p in zip(unit, ph.enter(xs)):
-            t = F.f32(P4_RANGE * F.f32(p))
-            pc, psf = F.nvfp4_quantize(t, axis=-1, block=16)
-            vt = F.nvfp4_dequantize(prep["v_f4"][kb], prep["v_sf4"][kb])
-            ph.acc += F.nvfp4_dequantize(pc, psf) @ vt.T
-    ph.fold_into(st, prep["v_g4"][None, :] / P4_RANGE)
+            x = np.where(valid[kb][None, :], (qd @ kd.T) * (inv_sqrt_d * LOG2E), -np.inf)
+            r_blk, w = p4_weights(x)
+            vt = F.nvfp4_dequantize(prep["v_f4"][kb], prep["v_sf4"][kb])  # [d, S] without g
+            ph.merge(r_blk * LN2, w.sum(1), w @ vt.T)
+        st.merge(ph.m, ph.l, ph.o * prep["v_g4"][None, :])
 
     out = np.where(st.l[:, None] > 0, st.o / np.where(st.l > 0, st.l, 1.0)[:, None], 0.0)
     return bf16_round(out) if mode == "emulate" else out
-
-
-def partner_of(prec_map, qb):
-    """Precision row of the other query block of qb's pair (2p, 2p+1), or None."""
-    o = qb ^ 1
-    return prec_map[o] if o < len(prec_map) else None
 
 
 def head_attention(prep, prec_map, d, mode="emulate", qblocks=None):
@@ -247,7 +186,7 @@ def head_attention(prep, prec_map, d, mode="emulate", qblocks=None):
     nb, S = prep["valid"].shape
     out = np.zeros((nb, S, d))
     for qb in (range(nb) if qblocks is None else qblocks):
-        out[qb] = qblock_attention(prep, qb, prec_map[qb], d, mode, partner_of(prec_map, qb))
+        out[qb] = qblock_attention(prep, qb, prec_map[qb], d, mode)
     return out
 
 
@@ -271,7 +210,7 @@ def dense_attention(q, k, v):
     return (p @ v) / p.sum(1, keepdims=True)
 
 
-def error_terms(prep, prec_map, d, qblocks, partner=True):
+def error_terms(prep, prec_map, d, qblocks):
     """Error decomposition of the method on the given query blocks of one head
     (DraftAttention2 abstract and reading note, Method overview: sparsity and
     quantisation are the two approximations; here they are measured apart).
@@ -287,8 +226,7 @@ def error_terms(prep, prec_map, d, qblocks, partner=True):
     num_s = num_q = num_t = den = 0.0
     for qb in qblocks:
         row = prec_map[qb]
-        other = partner_of(prec_map, qb) if partner else None
-        mixed = qblock_attention(prep, qb, row, d, "math", other)
+        mixed = qblock_attention(prep, qb, row, d, "math")
         exact_row = np.where(np.isin(row, list(kept)), BIT16, 0).astype(row.dtype)
         sparse = qblock_attention(prep, qb, exact_row, d, "math")
         dense = qblock_attention(prep, qb, np.full_like(row, BIT16), d, "math")

@@ -150,7 +150,7 @@ def oracle_rows(op, pr, prec_map, qblocks, mode="emulate"):
     tab = pr["table"]
     toks, rows = [], []
     for qb in qblocks:
-        o = OA.qblock_attention(pr, qb, prec_map[qb], op.d, mode, OA.partner_of(prec_map, qb))
+        o = OA.qblock_attention(pr, qb, prec_map[qb], op.d, mode)
         ok = tab[qb] >= 0
         toks.append(tab[qb][ok])
         rows.append(o[ok])
