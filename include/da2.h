@@ -46,7 +46,8 @@ extern "C" {
 enum {
   DA2_OK = 0,
   DA2_ERR_ARG = 1,          /* invalid sizes, pointers, lambda or budget       */
-  DA2_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, rh*rw != 64, no sm_100 GPU    */
+  DA2_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, rh*rw != 64, no sm_100 GPU,
+                               no TMA tensor-map encoder in the driver          */
   DA2_ERR_WORKSPACE = 3,    /* workspace NULL, misaligned or too small         */
   DA2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed            */
   DA2_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (see below)  */
@@ -99,38 +100,64 @@ int da2_prepare(const da2_problem* p, const void* q, const void* k, const void* 
  * per head over region pairs (fp32), then one ranking per head, descending by D
  * with ties broken by ascending pair index q_block*nb + k_block, hands out the
  * budget: first n16 pairs 16-bit, next n8 INT8, next n4 NVFP4, rest skipped.
+ * Also builds, per pair of neighbouring query blocks (2p, 2p+1), the merged
+ * key lists the attention kernel walks.
  * Requires da2_prepare on the same workspace first. */
 int da2_draft_rank(const da2_problem* p, void* ws, size_t ws_bytes, void* stream);
 
-/* Test hook for stage 2: ranking and assignment only, on caller-given fp32
- * scores [B,H,nb,nb] (device), which are copied into the workspace first. */
+/* Test hook for stage 2: ranking, assignment and the pair lists only, on
+ * caller-given fp32 scores [B,H,nb,nb] (device), which are copied into the
+ * workspace first. */
 int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
                          size_t ws_bytes, void* stream);
 
-/* Stage 3 ([abstract]; [note] Method overview bullet 4; [v1] order restore).
+/* Stage 3 ([abstract]; [note] Method overview bullets 3-4; [v1] order restore).
  * Per query block one pass runs the 16-bit phase (bf16 Q/K/V), the INT8 phase
  * and the NVFP4 phase over its assigned key blocks with one shared online
- * softmax state and one fp32 output accumulator.  Key blocks are taken two at
- * a time over the merged lists of the query-block pair (2p, 2p+1); low-bit P
- * is quantised against a running power of two per row and phase, raised per
- * such unit to the ceiling of the unit's row maximum (4-bit P as NVFP4 of
- * 2688 p), and each low-bit phase joins the shared accumulator with its
- * channel scale at the phase boundary.  The output rows are written straight
- * back to the original token order (padding rows dropped); a query block with
- * no key block outputs zeros.
+ * softmax state and one fp32 output accumulator.  Low-bit P is quantised per
+ * (query row, key block) against that block's own row maximum: INT8 codes
+ * round(255 exp(s - m_blk)); NVFP4 of 2688 * 2^(x - ceil(max x)) per 16 keys
+ * (x = s log2 e).  Each low-bit block enters numerator and row sum with the
+ * same quantised weights, and each phase joins the shared accumulator with
+ * its V channel scale.  The output rows are written straight back to the
+ * original token order (padding rows dropped); a query block with no key
+ * block outputs zeros.
  * q, k, v: the same device tensors given to da2_prepare; out: device bf16
- * [B,H,N,d].  Requires da2_draft_rank (or da2_rank_from_scores) first. */
+ * [B,H,N,d].  Requires da2_draft_rank (or da2_rank_from_scores) first.
+ * Every wait inside the kernel is bounded: read the outcome with
+ * da2_check_status.  Returns DA2_ERR_UNSUPPORTED when the driver lacks the
+ * TMA tensor-map encoder the kernel needs (there is no other kernel). */
 int da2_attention(const da2_problem* p, const void* q, const void* k, const void* v,
                   void* ws, size_t ws_bytes, void* out, void* stream);
 
 /* Own dense bf16 softmax attention over all N tokens (the comparison point
  * for the sparse path): out = softmax(q k^T / sqrt d) v, fp32 accumulation,
- * bf16 output.  q, k, v, out: device bf16 [B,H,N,d]; d in {64,128}.  For
- * d = 128 (N >= 64, B*H <= 65535) it runs the sparse path's tensor-core
+ * bf16 output.  q, k, v, out: device bf16 [B,H,N,d]; d in {64,128}, N >= 64
+ * (otherwise DA2_ERR_UNSUPPORTED).  It runs the sparse path's tensor-core
  * kernel with every key block in the 16-bit phase, over 64-token blocks in
- * natural order; otherwise a warp-MMA kernel.  Needs no workspace. */
+ * natural order.  Needs no workspace; its bounded-wait status goes to a word
+ * inside the library, read with da2_dense_check_status.  No counterpart on
+ * the pages beyond dense attention itself. */
 int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k,
                         const void* v, void* out, void* stream);
+
+/* Status of the dense calls on the current device since the last
+ * da2_dense_attention was enqueued: synchronises `stream`, returns DA2_OK, or
+ * DA2_ERR_TIMEOUT if a bounded wait in a dense kernel expired (its output is
+ * then incomplete), or DA2_ERR_CUDA.  Dense calls share the word, so
+ * concurrent dense calls on one device report together. */
+int da2_dense_check_status(void* stream);
+
+/* Test hook for the failure path, no counterpart on the pages: runs
+ * da2_attention with every bounded wait limited to `wait_polls` polls and
+ * with CTA `withheld_cta` (blockIdx.x; -1 for none) never issuing its first
+ * key-tile load, so that the waits on that tile run out.  The kernel then
+ * raises the workspace status word, stops issuing work, waits (bounded) for
+ * its copies in flight and releases its tensor memory; da2_check_status
+ * returns DA2_ERR_TIMEOUT.  Nothing faults and the context stays usable. */
+int da2_attention_wait_test(const da2_problem* p, const void* q, const void* k, const void* v,
+                            void* ws, size_t ws_bytes, void* out, int withheld_cta,
+                            unsigned int wait_polls, void* stream);
 
 /* Workspace views for tests.  Returns the device address and size of one
  * intermediate inside `ws` (no device work).  Layouts (bh = b*H + h):
@@ -183,8 +210,9 @@ int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t
  * DA2_NOALLOC_MAX_HEADS (batch x head) pairs; larger problems return
  * DA2_ERR_UNSUPPORTED before any device work.  Every GPU that loads the
  * library keeps that array (about 1.5 MB) until the process exits.  The first
- * call on a device looks the array's device address up (a runtime call); make
- * that first call before any stream capture.  Calls on one device share the
+ * call on a device (and the first after that device's context was reset)
+ * looks the array's device address up (a runtime call) and keeps it for that
+ * context; make that first call before any stream capture.  Calls on one device share the
  * array: calls that may overlap on the GPU (different streams, no ordering)
  * race and give wrong results; serialise them.  No call depends on what an
  * earlier call left in the array.  The call allocates nothing: no cudaMalloc,
@@ -193,7 +221,6 @@ int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t
 int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, uint16_t* lists,
                      int32_t* counts, void* stream);
 
-/* Human-readable name of a status code (static string). */
 /* Device status of the last da2_attention on `ws`: synchronises `stream`, reads
  * the workspace status word and returns DA2_OK, or DA2_ERR_TIMEOUT if a
  * bounded wait inside the attention kernel expired (the call's output is then
@@ -227,6 +254,7 @@ int da2_host_bytes(const da2_problem* p, int heads_per_chunk, size_t* bytes);
 int da2_forward_host(const da2_problem* p, const void* q, const void* k, const void* v, void* out,
                      void* dev, size_t dev_bytes, int heads_per_chunk, void* stream);
 
+/* Human-readable name of a status code (static string). */
 const char* da2_status_string(int status);
 
 #ifdef __cplusplus

@@ -68,7 +68,11 @@ int check_ws(const Layout& L, const void* ws, size_t ws_bytes) {
 
 bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
+// cudaErrorNotSupported is what the launchers return for a problem or driver
+// the kernels do not cover (no fallback kernel exists).
+int cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? DA2_OK : (e == cudaErrorNotSupported ? DA2_ERR_UNSUPPORTED : DA2_ERR_CUDA);
+}
 
 // Host-buffer path: the (batch, head) slices run in chunks of G, each chunk a
 // problem of its own (B = 1, H = chunk size; every stage is per head).  Two
@@ -149,6 +153,8 @@ int da2_draft_rank(const da2_problem* p, void* ws, size_t ws_bytes, void* stream
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = launch_draft(g, L, ws, st);
   if (e == cudaSuccess) e = launch_rank(g, L, ws, /*hist0_done=*/true, st);
+  // the attention kernel walks query blocks in pairs: their merged key lists
+  if (e == cudaSuccess) e = launch_pair_lists(g, L, ws, st);
   return cuda_status(e);
 }
 
@@ -165,6 +171,7 @@ int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
   cudaError_t e = cudaMemcpyAsync(at<float>(ws, L, R_SCORES), scores, L.size[R_SCORES],
                                   cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = launch_rank(g, L, ws, /*hist0_done=*/false, st);
+  if (e == cudaSuccess) e = launch_pair_lists(g, L, ws, st);
   return cuda_status(e);
 }
 
@@ -183,12 +190,34 @@ int da2_attention(const da2_problem* p, const void* q, const void* k, const void
 int da2_dense_attention(int B, int H, int N, int d, const void* q, const void* k,
                         const void* v, void* out, void* stream) {
   if (B <= 0 || H <= 0 || N <= 0) return DA2_ERR_ARG;
-  if (d != 64 && d != 128) return DA2_ERR_UNSUPPORTED;
+  if ((d != 64 && d != 128) || N < 64) return DA2_ERR_UNSUPPORTED;
   if ((long long)B * H > (1LL << 20) || N > (1 << 30)) return DA2_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DA2_ERR_ARG;
   int rc = check_device();
   if (rc) return rc;
   return cuda_status(launch_dense(B, H, N, d, q, k, v, out, (cudaStream_t)stream));
+}
+
+int da2_dense_check_status(void* stream) {
+  int rc = check_device();
+  if (rc) return rc;
+  int word = 0;
+  if (dense_status(&word, (cudaStream_t)stream) != cudaSuccess) return DA2_ERR_CUDA;
+  return word ? DA2_ERR_TIMEOUT : DA2_OK;
+}
+
+int da2_attention_wait_test(const da2_problem* p, const void* q, const void* k, const void* v,
+                            void* ws, size_t ws_bytes, void* out, int withheld_cta,
+                            unsigned int wait_polls, void* stream) {
+  Geom g;
+  int rc = make_geom(p, &g);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || wait_polls == 0) return DA2_ERR_ARG;
+  const Layout L = make_layout(g);
+  if ((rc = check_ws(L, ws, ws_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  return cuda_status(launch_attention_test(g, L, q, k, v, ws, out, (cudaStream_t)stream, wait_polls,
+                                           withheld_cta));
 }
 
 int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes) {
@@ -320,7 +349,7 @@ const char* da2_status_string(int s) {
     case DA2_ERR_UNSUPPORTED: return "unsupported problem or device";
     case DA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case DA2_ERR_CUDA: return "CUDA launch or runtime error";
-    case DA2_ERR_TIMEOUT: return "a bounded wait in the attention kernel expired";
+    case DA2_ERR_TIMEOUT: return "a bounded wait in an attention kernel expired";
     default: return "unknown status";
   }
 }

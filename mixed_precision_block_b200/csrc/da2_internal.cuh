@@ -184,18 +184,19 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
                              const void* v, void* ws, void* out, cudaStream_t st);
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k,
                          const void* v, void* out, cudaStream_t st);
+// Status word of the dense path: synchronises `st` and copies it to *word.
+cudaError_t dense_status(int* word, cudaStream_t st);
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st);
 // TMA: whether the driver's tensor-map encoder was found, and the 4-D view
 // [B*H*T][Hh][Ww][d] of a bf16 [B,H,N,d] tensor in {64 channels, rw, rh, 1}
 // region boxes (zero fill outside the frame).
 bool tma_available();
-bool dense_tc_supported(int B, int H, int N, int d);
-cudaError_t launch_dense_tc(int B, int H, int N, const void* q, const void* k, const void* v, void* out,
-                            cudaStream_t st);
 bool make_region_map(CUtensorMap* m, const void* base, const Geom& g, bool swizzle128);
-bool attention_tc_supported(const Geom& g);
-cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, const void* k,
-                                const void* v, void* ws, void* out, cudaStream_t st);
+// The attention kernel with an explicit wait bound (polls) and a CTA whose
+// first key load is withheld (-1: none), for the failure-path test.
+cudaError_t launch_attention_test(const Geom& g, const Layout& L, const void* q, const void* k,
+                                  const void* v, void* ws, void* out, cudaStream_t st,
+                                  uint32_t spin, int poison);
 cudaError_t launch_rank_noalloc(const Geom& g, const float* scores, uint8_t* map, uint16_t* lists,
                                 int* counts, cudaStream_t st);
 }  // namespace da2

@@ -18,6 +18,8 @@
 //                the per-query-block key lists (ballot/popc compaction)
 #include <mutex>
 
+#include <cuda.h>
+
 #include "da2_internal.cuh"
 
 namespace da2 {
@@ -413,22 +415,52 @@ static __device__ __align__(256) unsigned char g_rank_scratch[kNoallocBytes];
 
 namespace {
 std::mutex g_scratch_mu;
-void* g_scratch_addr[64];  // device address of g_rank_scratch, per device ordinal
+void* g_scratch_addr[64];                // device address of g_rank_scratch, per device ordinal
+unsigned long long g_scratch_ctx[64];    // id of the context that address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (0 if unknown).  A
+// context created after cudaDeviceReset gets a new id, so an address cached
+// for the old context is never reused.
+unsigned long long current_ctx_id() {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // In host code `g_rank_scratch` names a host-side shadow, not device memory:
-// the device address has to be looked up once per device, with that device
-// current, before a kernel can be given it.
+// the device address has to be looked up, with the device current, before a
+// kernel can be given it.  That happens once per device and context (the
+// first call on a device, and the first call after its context was reset).
 cudaError_t rank_scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long id = current_ctx_id();
+  if (!g_scratch_addr[dev] || id == 0 || id != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_rank_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_ctx_id();  // the lookup made the context current
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

@@ -4,17 +4,17 @@
 // Figure 3(b)): Q/K reordering, pooling and quantisation share one kernel;
 // V is reordered and transposed while it is packed.
 //
-// prep_qk: one CTA per (region block, head, tensor Q|K).  The block's 64 tokens
-//   are 8 rows of 8 consecutive tokens in the [B,H,N,d] input, so each token
-//   is one contiguous d*2-byte row; 256 threads read it in 16-byte chunks
-//   (coalesced 128-bit loads, padding slots are never read).  In one pass the
-//   CTA produces the pooled mean / max (warp-shuffle + shared-memory
-//   reductions), the INT8 codes with the block's absmax scale, and the NVFP4
-//   codes with one e4m3 scale per 16 channels of a token.
-// v_amax + pack_v: the per-channel absmax of V over all real tokens of a head
-//   (first pass, atomicMax on the float bits), then one CTA per block that
-//   stages the block transposed in shared memory and writes INT8 and NVFP4
-//   codes in [block][channel][token] order.
+// prep_qk_tma: persistent; each CTA walks (tensor Q|K, head, region block)
+//   items, one thread keeping a ring of region tiles in flight with TMA (an
+//   8x8-token box per 64 channels straight from the [B,H,N,d] input, zero
+//   outside the frame).  From shared memory the CTA produces the pooled mean /
+//   max (warp-shuffle + shared-memory reductions), the INT8 codes with the
+//   block's absmax scale, and the NVFP4 codes with one e4m3 scale per 16
+//   channels of a token.
+// v_amax + pack_v_tma: the per-channel absmax of V over all real tokens of a
+//   head (first pass, atomicMax on the float bits), then the same TMA ring
+//   over V's region tiles, which writes INT8 and NVFP4 codes in
+//   [block][channel][token] order.
 #include "da2_internal.cuh"
 #include "sm100.cuh"
 
@@ -44,15 +44,6 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   }
 }
 
-// Number of real tokens in a region block.
-__device__ __forceinline__ int block_real_count(const Geom& g, int blk) {
-  const int rx = blk % g.nrx;
-  const int ry = (blk / g.nrx) % g.nry;
-  const int ny = min(g.rh, g.Hh - ry * g.rh);
-  const int nx = min(g.rw, g.Ww - rx * g.rw);
-  return ny * nx;
-}
-
 __device__ __forceinline__ uint32_t quant_i8x4(const float* x, float inv) {
   uint32_t r = 0;
 #pragma unroll
@@ -80,113 +71,6 @@ __device__ __forceinline__ uint32_t quant_f4x8(const float* x, float amax16, uin
     out |= b << (8 * m);
   }
   return out;
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads) prep_qk_kernel(Geom g, PrepPtrs P, int want_i8,
-                                                           int want_f4) {
-  constexpr int CPT = D / 8;                // 16-byte chunks per token
-  constexpr int NC = 64 * CPT / kThreads;   // chunks per thread
-  constexpr int SLOT_STEP = kThreads / CPT;
-  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int cg = tid % CPT, slot0 = tid / CPT;
-  const __nv_bfloat16* __restrict__ x = P.x[which] + (size_t)bh * g.N * D;
-
-  float v[NC][8];
-  bool valid[NC];
-#pragma unroll
-  for (int i = 0; i < NC; ++i) {
-    const int s = slot0 + i * SLOT_STEP;
-    const int tok = slot_token(g, blk, s);
-    valid[i] = tok >= 0;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (valid[i]) u = *reinterpret_cast<const uint4*>(x + (size_t)tok * D + cg * 8);
-    unpack8(u, v[i]);
-  }
-  if (which == 0 && bh == 0 && tid < 64) P.perm[blk * 64 + tid] = slot_token(g, blk, tid);
-
-  // ---- pooled mean and max over real tokens
-  float psum[8], pmax[8], amax = 0.f;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) { psum[c] = 0.f; pmax[c] = -INFINITY; }
-#pragma unroll
-  for (int i = 0; i < NC; ++i) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      if (valid[i]) { psum[c] += v[i][c]; pmax[c] = fmaxf(pmax[c], v[i][c]); }
-      amax = fmaxf(amax, fabsf(v[i][c]));
-    }
-  }
-  // lanes sharing a channel group differ in the bits at and above log2(CPT)
-#pragma unroll
-  for (int o = CPT; o < 32; o <<= 1) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      psum[c] += __shfl_xor_sync(0xffffffffu, psum[c], o);
-      pmax[c] = fmaxf(pmax[c], __shfl_xor_sync(0xffffffffu, pmax[c], o));
-    }
-  }
-  __shared__ float s_sum[kThreads / 32][D];
-  __shared__ float s_max[kThreads / 32][D];
-  __shared__ float s_amax[kThreads / 32];
-  if (lane < CPT) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      s_sum[warp][cg * 8 + c] = psum[c];
-      s_max[warp][cg * 8 + c] = pmax[c];
-    }
-  }
-  amax = warp_max(amax);
-  if (lane == 0) s_amax[warp] = amax;
-  __syncthreads();
-  const size_t blk_lin = (size_t)bh * g.nb + blk;
-  if (tid < D) {
-    float s = 0.f, m = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) { s += s_sum[w][tid]; m = fmaxf(m, s_max[w][tid]); }
-    P.avg[which][blk_lin * D + tid] = s / (float)block_real_count(g, blk);
-    P.mx[which][blk_lin * D + tid] = m;
-  }
-  amax = s_amax[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, s_amax[w]);
-
-  // ---- INT8: one symmetric scale per block
-  if (want_i8) {
-    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-    if (tid == 0) P.s8[which][blk_lin] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
-    int8_t* __restrict__ dst = P.i8[which] + blk_lin * 64 * D;
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-      const int s = slot0 + i * SLOT_STEP;
-      uint2 w;
-      w.x = quant_i8x4(v[i], inv);
-      w.y = quant_i8x4(v[i] + 4, inv);
-      *reinterpret_cast<uint2*>(dst + (size_t)s * D + cg * 8) = w;
-    }
-  }
-  // ---- NVFP4: e4m3 scale per 16 channels of a token
-  if (want_f4) {
-    uint8_t* __restrict__ dst = P.f4[which] + blk_lin * 64 * (D / 2);
-    uint8_t* __restrict__ sfd = P.sf4[which] + blk_lin * (D / 64) * kSfAtomBytes;
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-      const int s = slot0 + i * SLOT_STEP;
-      float a8 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) a8 = fmaxf(a8, fabsf(v[i][c]));
-      const float a16 = fmaxf(a8, __shfl_xor_sync(0xffffffffu, a8, 1));
-      uint32_t sfb;
-      const uint32_t codes = quant_f4x8(v[i], a16, &sfb);
-      *reinterpret_cast<uint32_t*>(dst + (size_t)s * (D / 2) + cg * 4) = codes;
-      if ((cg & 1) == 0) {
-        const int o = sf_atom_offset(s, cg / 2);
-        sfd[o] = (uint8_t)sfb;
-        sfd[o + 8] = (uint8_t)sfb;  // rows 64..127 of the atom repeat rows 0..63
-      }
-    }
-  }
 }
 
 // bytes 0 of four words -> one word (x0 in the low byte)
@@ -421,67 +305,6 @@ struct VPtrs {
   float* g4;
 };
 
-template <int D>
-__global__ void __launch_bounds__(kThreads) pack_v_kernel(Geom g, VPtrs P, int want_i8, int want_f4) {
-  constexpr int CPT = D / 8;
-  constexpr int NC = 64 * CPT / kThreads;
-  constexpr int SLOT_STEP = kThreads / CPT;
-  const int blk = blockIdx.x, bh = blockIdx.y;
-  const int tid = threadIdx.x;
-  const int cg = tid % CPT, slot0 = tid / CPT;
-  __shared__ float s_v[D][65];  // transposed tile [channel][slot], +1 against bank conflicts
-  const __nv_bfloat16* __restrict__ x = P.v + (size_t)bh * g.N * D;
-#pragma unroll
-  for (int i = 0; i < NC; ++i) {
-    const int s = slot0 + i * SLOT_STEP;
-    const int tok = slot_token(g, blk, s);
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (tok >= 0) u = *reinterpret_cast<const uint4*>(x + (size_t)tok * D + cg * 8);
-    float f[8];
-    unpack8(u, f);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) s_v[cg * 8 + c][s] = f[c];
-  }
-  __syncthreads();
-  const size_t blk_lin = (size_t)bh * g.nb + blk;
-  const unsigned int* amax_bits = P.amax_bits + (size_t)bh * D;
-  if (blk == 0 && tid < D) {
-    const float a = __uint_as_float(amax_bits[tid]);
-    if (want_i8) P.s8[(size_t)bh * D + tid] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
-    if (want_f4) P.g4[(size_t)bh * D + tid] = __fdiv_rn(a, 2688.0f);
-  }
-  // items: (channel c, 16-slot group j); 4 groups per channel
-  for (int item = tid; item < D * 4; item += kThreads) {
-    const int c = item >> 2, j = item & 3;
-    const float a = __uint_as_float(amax_bits[c]);
-    float f[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) f[e] = s_v[c][16 * j + e];
-    if (want_i8) {
-      const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
-      uint4 w;
-      w.x = quant_i8x4(f, inv);
-      w.y = quant_i8x4(f + 4, inv);
-      w.z = quant_i8x4(f + 8, inv);
-      w.w = quant_i8x4(f + 12, inv);
-      *reinterpret_cast<uint4*>(P.i8 + (blk_lin * D + c) * 64 + 16 * j) = w;
-    }
-    if (want_f4) {
-      const float gch = __fdiv_rn(a, 2688.0f);
-      const float r = gch > 0.f ? __fdiv_rn(1.0f, gch) : 0.f;
-      float a16 = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) { f[e] = __fmul_rn(f[e], r); a16 = fmaxf(a16, fabsf(f[e])); }
-      uint32_t sfb;
-      uint2 w;
-      w.x = quant_f4x8(f, a16, &sfb);
-      w.y = quant_f4x8(f + 8, a16, &sfb);
-      *reinterpret_cast<uint2*>(P.f4 + (blk_lin * D + c) * 32 + 8 * j) = w;
-      P.sf4[blk_lin * kSfAtomBytes + sf_atom_offset(c, j)] = (uint8_t)sfb;
-    }
-  }
-}
-
 // pack_v_tma: persistent form of pack_v with the same TMA ring as
 // prep_qk_tma.  The tile stays as loaded ([slot][channel], bf16); a thread
 // takes two neighbouring channels of one 16-slot group, reads them down the
@@ -615,7 +438,7 @@ cudaError_t launch_prepare_d(const Geom& g, const Layout& L, const void* q, cons
     const int grid = std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
     prep_qk_tma_kernel<D><<<grid, kThreads, LY::TOTAL, st>>>(tq, tk, g, P, want_i8, want_f4, n_items);
   } else {
-    prep_qk_kernel<D><<<dim3(g.nb, g.BH, 2), kThreads, 0, st>>>(g, P, want_i8, want_f4);
+    return cudaErrorNotSupported;  // no tensor-map encoder in this driver
   }
   e = cudaGetLastError();
   if (e != cudaSuccess || !(want_i8 || want_f4)) return e;
@@ -643,7 +466,7 @@ cudaError_t launch_prepare_d(const Geom& g, const Layout& L, const void* q, cons
     const int grid = std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
     pack_v_tma_kernel<D><<<grid, kThreads, LY::TOTAL, st>>>(tv, g, V, want_i8, want_f4, n_items);
   } else {
-    pack_v_kernel<D><<<dim3(g.nb, g.BH), kThreads, 0, st>>>(g, V, want_i8, want_f4);
+    return cudaErrorNotSupported;  // no tensor-map encoder in this driver
   }
   return cudaGetLastError();
 }

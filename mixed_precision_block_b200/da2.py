@@ -26,8 +26,8 @@ VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_
          "Q_F4", "K_F4", "Q_SF4", "K_SF4", "V_I8", "V_S8", "V_F4", "V_SF4", "V_G4",
          "SCORES", "MAP", "LISTS", "COUNTS", "STATUS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
-           "da2_dense_attention", "da2_debug_view", "da2_rank_noalloc", "da2_check_status",
-           "da2_host_bytes", "da2_forward_host", "da2_status_string"]
+           "da2_dense_attention", "da2_dense_check_status", "da2_attention_wait_test", "da2_debug_view",
+           "da2_rank_noalloc", "da2_check_status", "da2_host_bytes", "da2_forward_host", "da2_status_string"]
 NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
 
 
@@ -64,6 +64,8 @@ _lib.da2_draft_rank.argtypes = [_P, _vp, _sz, _vp]
 _lib.da2_rank_from_scores.argtypes = [_P, _vp, _vp, _sz, _vp]
 _lib.da2_attention.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.da2_dense_attention.argtypes = [ctypes.c_int] * 4 + [_vp] * 5
+_lib.da2_dense_check_status.argtypes = [_vp]
+_lib.da2_attention_wait_test.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, ctypes.c_int, ctypes.c_uint, _vp]
 _lib.da2_debug_view.argtypes = [_P, _vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]
 _lib.da2_rank_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
 _lib.da2_check_status.argtypes = [_P, _vp, _sz, _vp]
@@ -177,6 +179,23 @@ def da2_dense_attention(q, k, v, out, stream=None):
     B, H, N, d = q.shape
     _check("da2_dense_attention", _lib.da2_dense_attention(B, H, N, d, _ptr(q), _ptr(k), _ptr(v),
                                                            _ptr(out), _stream(stream, q)))
+
+
+def da2_dense_check_status(stream=None):
+    """Synchronise `stream` and return the dense calls' status (0, or
+    DA2_ERR_TIMEOUT = 5 if a bounded wait in a dense kernel expired)."""
+    return _lib.da2_dense_check_status(_vp(stream if isinstance(stream, int) else
+                                           (stream.cuda_stream if stream is not None
+                                            else torch.cuda.current_stream().cuda_stream)))
+
+
+def da2_attention_wait_test(p, q, k, v, ws, out, withheld_cta, wait_polls, stream=None):
+    """Failure-path test hook: da2_attention with every wait bounded by
+    `wait_polls` polls and CTA `withheld_cta` never issuing its first key
+    load.  Returns the call's status code (the kernel's own outcome is read
+    with da2_check_status)."""
+    return _lib.da2_attention_wait_test(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel(),
+                                        _ptr(out), int(withheld_cta), int(wait_polls), _stream(stream, ws))
 
 
 def da2_debug_view(p, ws, which):

@@ -67,23 +67,26 @@ def test_reference_arm_is_rank_zero_only(monkeypatch):
     assert buf.getvalue() == ""
 
 
-def test_roofline_takes_the_larger_floor():
+def test_roofline_follows_the_phase_floors_and_prep_bytes():
     sys.path.insert(0, ROOT)
     import bench
     from types import SimpleNamespace
     from mixed_precision_block_b200.synth import WORKLOADS
-    pk = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
-    wl = WORKLOADS["video"]  # 24 heads
-    # 16-bit only: tensor floor = 4*64*64*128 FLOP * n16 * 24 / 1.4e15; XU = 6144 ops * n16 * 24 / (16*148*1965e6)
-    info = SimpleNamespace(n16=1000, n8=0, n4=0)
-    r = bench.attention_roofline(wl, info, 1.0, pk, "measured", 1965.0)
-    t_tensor = 4 * 64 * 64 * 128 * 1000 * 24 / 1.4e15 * 1e3
-    t_xu = 6144 * 1000 * 24 / (16 * 148 * 1965e6) * 1e3
-    assert abs(r["floors_ms"]["tensor"] - t_tensor) < 1e-12 and abs(r["floors_ms"]["xu"] - t_xu) < 1e-12
-    assert r["bound"] == ("tensor" if t_tensor >= t_xu else "alu")
-    assert abs(r["frac"] - max(t_tensor, t_xu) / 1.0) < 1e-12  # achieved/peak = floor/time
-    # 4-bit only: the tensor floor is a quarter, the XU floor larger: bound by the XU pipe
-    info = SimpleNamespace(n16=0, n8=0, n4=1000)
-    r = bench.attention_roofline(wl, info, 1.0, pk, "measured", 1965.0)
-    assert r["bound"] == "alu" and r["unit"] == "Gop/s"
+    pk = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    wl = WORKLOADS["video"]  # 24 heads, d = 128, 118,800 tokens, 1980 regions
+    # the survey's worked figure for the headline budget: 3.46 GB of prep traffic
+    info = SimpleNamespace(n16=294030, n8=294030, n4=0, nb=1980)
+    assert abs(bench.prep_bytes(wl, info) / 1e9 - 3.46) < 0.01
+    # phase floors: 16-bit at the burst bf16 peak, INT8 at twice it, NVFP4 at four times
+    info = SimpleNamespace(n16=1000, n8=2000, n4=4000, nb=1980)
+    r = bench.roofline(wl, info, 2.0, 4.0, pk, "measured", 1965.0)
+    per_pair = 4 * 64 * 64 * 128 * 24
+    t_tensor = (1000 * per_pair / 1.6e15 + 2000 * per_pair / 3.2e15 + 4000 * per_pair / 6.4e15) * 1e3
+    assert abs(r["floor_ms"]["tensor"] - t_tensor) < 1e-12
+    assert abs(r["frac"] - t_tensor / 2.0) < 1e-12  # achieved / phase-weighted peak = floor / time
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    t_prep = bench.prep_bytes(wl, info) / 6.5e12 * 1e3
+    assert abs(r["whole_call"]["frac"] - (t_tensor + t_prep) / 4.0) < 1e-12
+    # the XU floor is reported beside it, not as the bound
+    t_xu = 24 * (1000 * 6144 + 2000 * 4096 + 4000 * 4096 * (1.5 + 1 / 16)) / (16 * 148 * 1965e6) * 1e3
+    assert r["bound"] == "tensor" and abs(r["xu_floor_ms"] - t_xu) < 1e-9
