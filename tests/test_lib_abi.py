@@ -86,6 +86,11 @@ def test_entry_points_check_workspace_and_pointers_before_launch(da2):
     assert lib.da2_attention(ctypes.byref(p), fake, fake, fake, fake, big, None, None) == da2.DA2_ERR_ARG
     assert lib.da2_dense_attention(1, 1, 64, 96, fake, fake, fake, fake, None) == da2.DA2_ERR_UNSUPPORTED
     assert lib.da2_dense_attention(1, 1, 0, 64, fake, fake, fake, fake, None) == da2.DA2_ERR_ARG
+    # one tensor-core kernel covers the dense path: shorter sequences than one
+    # 64-token block are refused, not sent to another kernel
+    assert lib.da2_dense_attention(1, 1, 63, 128, fake, fake, fake, fake, None) == da2.DA2_ERR_UNSUPPORTED
+    assert lib.da2_attention_wait_test(ctypes.byref(p), fake, fake, fake, fake, big, fake, 0, 0,
+                                       None) == da2.DA2_ERR_ARG  # a zero wait bound
     assert lib.da2_check_status(ctypes.byref(p), None, big, None) == da2.DA2_ERR_WORKSPACE
     assert lib.da2_check_status(ctypes.byref(p), fake, big - 1, None) == da2.DA2_ERR_WORKSPACE
 
