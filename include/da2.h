@@ -169,7 +169,9 @@ int da2_attention_wait_test(const da2_problem* p, const void* q, const void* k, 
  *          atom whose line i holds the 4 scales (16 channels each) of slots i
  *          and i+32 as two 32-bit words, repeated in words 2-3 (the layout the
  *          tensor core reads scale factors from)
- *   V_I8  int8 [B*H][nb][d][64];  V_S8 fp32 [B*H][d]
+ *   V_I8  bf16 [B*H][nb][64][d]: V's INT8 codes (integers -127..127, exact
+ *          as bf16) in block slot order, the operand layout of the P.V MMA;
+ *          V_S8 fp32 [B*H][d]
  *   V_F4  uint8 [B*H][nb][d][32] (even token in the low nibble)
  *   V_SF4 uint8 e4m3 [B*H][nb][32][16]: line i holds the 4 scales (16 tokens
  *          each) of channels i, i+32, i+64, i+96;  V_G4 fp32 [B*H][d]

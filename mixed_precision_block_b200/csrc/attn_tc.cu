@@ -14,8 +14,9 @@
 // rows 0-63 and 64-127 of one M = 128 tile — and walks the merged key list of
 // the pair phase by phase, two key blocks (a "unit") at a time.  A key block
 // only one of the two keeps is computed for all 128 rows and masked for the
-// other half.  Nothing a row computes depends on the other query block: every
-// quantisation reference below is the row's own.
+// other half.  Nothing a row computes depends on the other query block, nor on
+// the grouping into units, beyond rounding: every quantisation reference below
+// is the row's own per key block, and references are powers of two.
 //
 // Roles (12 warps).  Warps 0-7 do the softmax: warp w holds 16 tile rows,
 // 32(w&3) + 16(w>>2) + i, with two threads per row (lanes i and i+16), reading
@@ -28,28 +29,31 @@
 //
 //   16-bit  S = Q·[K_a;K_b]^T (kind::f16, fp32 in TMEM, two buffers);
 //           P = exp2(s·log2e/√d − m) rounded to bf16 against an integer
-//           reference m per row, raised lazily (O rescaled in TMEM only when
-//           the row max grows by more than 2^8); P replaces the scores in TMEM
-//           and O += P·V reads it from there (V MN-major from the TMA tile).
-//   8-bit   S8 = Q8·[K8_a;K8_b]^T (kind::i8, s32); per row and key block the
-//           reference is the block's own maximum: codes round(255 exp(s −
-//           m_blk)) replace the scores in TMEM; D_t = P8_t·V8_t (kind::i8
-//           u8×s8) goes to its own s32 accumulator per block, started from the
-//           bit pattern of 1.5·2^23 so that one float subtraction reads it
-//           exactly; the softmax threads fold each D_t into O, held in
-//           registers through the low-bit phases, with weight exp(m_blk − m);
-//           the row sum takes the code sums with the same weights.
+//           reference m per row (the shared statistics), raised lazily (O
+//           rescaled in TMEM only when the row max grows by more than 2^8); P
+//           replaces the scores in TMEM and O += P·V reads it from there (V
+//           MN-major from the TMA tile).
+//   8-bit   S8 = Q8·[K8_a;K8_b]^T (kind::i8, s32).  Per row and key block the
+//           reference is the block's own maximum rounded up to a power of two,
+//           2^r_blk: codes c = round(255·2^(x − r_blk)).  c·2^(r_blk − m) is an
+//           8-bit integer times a power of two, exact in bf16, and so are the
+//           INT8 V codes: O += P·V8 runs on the 16-bit path (kind::f16, P from
+//           TMEM) straight into the shared accumulator, every product exact.
+//           The row sum takes the same weights /255.
 //   4-bit   S = Q4·K4_t^T (kind::mxf4nvf4, block16 ue4m3 scales copied into
-//           TMEM with tcgen05.cp); P = NVFP4 of 2688·2^(x − r) per 16 keys
-//           against one power-of-two reference r per row, raised to the ceiling
-//           of a unit's maximum (which reproduces each block's own power-of-two
-//           reference while the microscale stays normal); O4 += P4·V4 in fp32
-//           TMEM, and L4 += P4·1 (an MMA against a tile of e2m1 ones) gives the
-//           row sum of the quantised weights.  O4 and L4 join O when r rises
-//           and at the end of the phase, with the channel scale g/2688.
+//           TMEM with tcgen05.cp); P = NVFP4 of 2688·2^(x − m) per 16 keys
+//           against the shared reference m, raised to the ceiling of the
+//           running maximum at the phase start and to a unit's maximum when
+//           it exceeds it (which reproduces each block's own power-of-two
+//           reference while the microscale stays normal); O += P4·V4 into the
+//           shared fp32 accumulator, and L4 += P4·1 (an MMA against a tile of
+//           e2m1 ones) gives the row sum of the quantised weights.
+//   Around each low-bit phase O is multiplied by the inverse of the phase's V
+//   channel scale (sv/255 or g/2688) and back — the rescaling at the phase
+//   boundaries — so that the phase's MMAs work on the codes.
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), codes as 2-D boxes of
-// the workspace.  The epilogue writes O / l through the same region box with a
+// the workspace (V's INT8 codes held as bf16 values by the preparation).  The epilogue writes O / l through the same region box with a
 // TMA store, whose clipping drops the padding rows — the restore.
 // Every wait is bounded; on expiry the CTA raises its status word, stops
 // issuing, waits (bounded) for its own copies in flight and releases its
@@ -90,13 +94,12 @@ constexpr uint32_t kOnesE2m1 = 0x22222222u;  // e2m1 1.0 in every nibble
 constexpr uint32_t kOneE4m3x4 = 0x38383838u; // ue4m3 1.0 in every byte
 constexpr uint32_t kDefaultSpin = 1u << 22;
 
-// TMEM columns (512 allocated).  [0, D): O in the 16-bit phase; in the INT8
-// phase the accumulator D_a of a unit's first key block (O moves to
-// registers); in the 4-bit phase the accumulator O4.  [128, 384): two score
-// buffers.  [384, 384+D): INT8 D_b.  4-bit phase: scale factors from 384 —
-// Q 384, K_a 392, K_b 400, V_a 408, V_b 412, P_a 416, P_b 420, ones 424 (all
-// 4-aligned, as block-scaled MMAs require) — and the row sums L4 at 448.
-constexpr uint32_t TM_O = 0, TM_S = 128, TM_DB = 384;
+// TMEM columns (512 allocated).  [0, D): O, the one fp32 accumulator every
+// phase adds into.  [128, 384): two score buffers.  4-bit phase: scale factors
+// from 384 — Q 384, K_a 392, K_b 400, V_a 408, V_b 412, P_a 416, P_b 420,
+// ones 424 (all 4-aligned, as block-scaled MMAs require) — and the row sums of
+// the quantised P, L4, at 448 (64 columns).
+constexpr uint32_t TM_O = 0, TM_S = 128;
 constexpr uint32_t TM_SFQ = 384, TM_SFK = 392, TM_SFV = 408, TM_SFP = 416, TM_SF1 = 424, TM_L4 = 448;
 
 // Shared-memory map (offsets from a 1024-aligned base).
@@ -113,8 +116,8 @@ struct Smem {
   static constexpr uint32_t P4STRIDE = 10240;              // P4_a 4 KB | P4_b 4 KB | SF_a | SF_b
   static constexpr uint32_t P4SF = 8192;
   static constexpr uint32_t ONES = P4 + 2 * P4STRIDE;      // [64 rows][32 B] of e2m1 1.0
-  static constexpr uint32_t VS = ONES + 2048;              // fp32 [3][D]: 255/sv, sv/255, g/2688
-  static constexpr uint32_t BAR = VS + ((12u * D + 255u) & ~255u);
+  static constexpr uint32_t VS = ONES + 2048;              // fp32 [4][D] channel factors (see VS_*)
+  static constexpr uint32_t BAR = VS + ((16u * D + 255u) & ~255u);
   static constexpr uint32_t MISC = BAR + 512;
   static constexpr uint32_t USED = MISC + 256;
   // ask for at least 120 KB so that one CTA holds an SM (it allocates all of TMEM)
@@ -125,9 +128,14 @@ struct Smem {
 static_assert(Smem<128>::BYTES <= 227 * 1024, "shared memory");
 static_assert(Smem<64>::BYTES <= 227 * 1024, "shared memory");
 
+// channel factors that move O into a low-bit phase's units and back:
+// 255/sv, sv/255 (INT8: V codes times sv/255... P codes /255), 2688/g, g/2688
+// (NVFP4: V/g and 2688 P); 1 where the channel scale is 0
+enum { VS_TO8 = 0, VS_FROM8 = 1, VS_TO4 = 2, VS_FROM4 = 3 };
+
 // mbarrier slots (8 bytes each)
 enum {
-  B_Q16 = 0, B_Q8, B_Q4, B_F4, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
+  B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
   B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages, B_P_FULL = B_S_FULL + 2,
   B_P_FREE = B_P_FULL + 2, B_DONE = B_P_FREE + 2, B_COUNT
 };
@@ -175,15 +183,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// bytes 0 of four words -> one word (x0 in the low byte)
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
-  uint32_t lo, hi, r;
-  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(x0), "r"(x1));
-  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(x2), "r"(x3));
-  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-// 2^k for an integer-valued float k <= 0 (exact; 0 below the normal range)
+// 2^k for an integer-valued float k <= 127 (exact; 0 below the normal range)
 __device__ __forceinline__ float pow2i(float k) { return k > -127.0f ? __int_as_float(((int)k + 127) << 23) : 0.0f; }
 
 // Items: kb | inA << 16 | inB << 17 | kind << 18 | full << 20 (the key block
@@ -239,7 +239,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC + 8);
   // 1 / (1 + m/8) for m = 0..7, then 1 / m (0 for m = 0): reciprocals of e4m3 scales
   float* rcp_tab = reinterpret_cast<float*>(smem + SM::MISC + 64);
-  float* vsc = reinterpret_cast<float*>(smem + SM::VS);  // [0,D) 255/sv, [D,2D) sv/255, [2D,3D) g/2688
+  float* vsc = reinterpret_cast<float*>(smem + SM::VS);  // [4][D] channel factors (VS_*)
   if (threadIdx.x < 16)
     rcp_tab[threadIdx.x] = threadIdx.x < 8 ? 8.0f / (float)(8 + threadIdx.x)
                                            : (threadIdx.x > 8 ? 1.0f / (float)(threadIdx.x - 8) : 0.f);
@@ -258,7 +258,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(bar(B_Q16), 1);
     mbar_init(bar(B_Q8), 1);
     mbar_init(bar(B_Q4), 1);
-    mbar_init(bar(B_F4), kSoftmaxWarps);
+    mbar_init(bar(B_SFQ), 4);  // warps 0-3 wrote Q's and the ones tile's scale factors
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(B_K_FULL + s), 1); mbar_init(bar(B_K_EMPTY + s), 1);
       mbar_init(bar(B_V_FULL + s), 1); mbar_init(bar(B_V_EMPTY + s), 1);
@@ -275,10 +275,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == kMmaWarp) tmem_alloc(s0 + SM::MISC, 512);
   if (!kDense) {
     for (int c = threadIdx.x; c < D; c += kThreads) {
-      const float sv = A.v_s8[(size_t)bh * D + c], gv = A.v_g4[(size_t)bh * D + c];
-      vsc[c] = sv > 0.f ? 255.0f / sv : 1.0f;
-      vsc[D + c] = sv > 0.f ? sv / 255.0f : 1.0f;
-      vsc[2 * D + c] = gv / kP4Range;
+      const float sv = n8 > 0 ? A.v_s8[(size_t)bh * D + c] : 0.f, gv = n4 > 0 ? A.v_g4[(size_t)bh * D + c] : 0.f;
+      vsc[VS_TO8 * D + c] = sv > 0.f ? 255.0f / sv : 1.0f;
+      vsc[VS_FROM8 * D + c] = sv > 0.f ? sv / 255.0f : 1.0f;
+      vsc[VS_TO4 * D + c] = gv > 0.f ? kP4Range / gv : 1.0f;
+      vsc[VS_FROM4 * D + c] = gv > 0.f ? gv / kP4Range : 1.0f;
     }
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + SM::ONES);
     for (int i = threadIdx.x; i < 512; i += kThreads) ones[i] = kOnesE2m1;
@@ -376,9 +377,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               for (int h = 0; h < H; ++h) tma_load_4d(dst + (t * H + h) * 8192, &tmV, fb, 64 * h, cx, cy, cf);
             }
           } else if (vn < nu8) {
-            mbar_expect_tx(fb, 64u * D * (uint32_t)cnt);
+            // the INT8 codes as bf16 values, [64 slots][D] per block: the 16-bit tile layout
+            mbar_expect_tx(fb, 128u * D * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t)
-              tma_load_2d(dst + t * 64 * D, &tmV8, fb, 0, (bh * g.nb + item_kb(item_at(i0 + t))) * D);
+              for (int h = 0; h < H; ++h)
+                tma_load_2d(dst + (t * H + h) * 8192, &tmV8, fb, 64 * h, (bh * g.nb + item_kb(item_at(i0 + t))) * 64);
           } else {
             mbar_expect_tx(fb, (32u * D + kSfAtomBytes) * (uint32_t)cnt);
             for (int t = 0; t < cnt; ++t) {
@@ -417,13 +420,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t idpv = idesc(kDF32, kFmtBF16, kFmtBF16, false, true, 128, D);
       const uint32_t id8n64 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
       const uint32_t id8n128 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 128);
-      const uint32_t idx8 = idesc(kDS32, kFmtU8, kFmtS8, false, false, 128, D);
       const uint32_t id4s = idesc_f4(128, 64), id4pv = idesc_f4(128, D), id4l = idesc_f4(128, 64);
       constexpr uint32_t kSbo8 = 8u * D;                       // INT8 rows of D bytes
       constexpr Swizzle kSw8 = D == 128 ? SW_128 : SW_64;
       constexpr uint32_t kSbo4 = 4u * D;                       // NVFP4 rows of D/2 bytes
       constexpr Swizzle kSw4 = D == 128 ? SW_64 : SW_32;
-      bool f4_ready = false;  // Q4 loaded, its scales in TMEM and the 4-bit TMEM area free
+      bool f4_ready = false;  // Q4 loaded and its scales in TMEM
       bool ok = true;
       if (n16 > 0) ok = ok && mbar_wait(bar(B_Q16), 0, spin);
       if (n8 > 0) ok = ok && mbar_wait(bar(B_Q8), 0, spin);
@@ -436,7 +438,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (sn < nu) {
           const int s = sn % kStages, b = sn & 1;
           const bool f4 = sn >= nu8;
-          if (f4 && !f4_ready) f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_F4), 0);
+          if (f4 && !f4_ready) f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
           // a score buffer is free once the P·V of the unit two back completed
           // (its P sat in the buffer, or its scores were read before its P)
           if ((!f4 || f4_ready) && pv_done(sn - 2) && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1)) {
@@ -485,20 +487,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const uint32_t pt = tbase + TM_S + (pn & 1) * 128u;  // the unit's P (16-bit, INT8) in TMEM
             int i0, cnt;
             unit_items(pn, i0, cnt);
-            if (pn < nu16) {
+            if (pn < nu8) {
+              // 16-bit and INT8 units: P (bf16) from TMEM, V tiles MN-major bf16
               for (int t = 0; t < cnt; ++t) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                   mma_f16_ta(tbase + TM_O, pt + 64 * t + 8 * kk,
                              smem_desc(st + t * H * 8192 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
-              }
-            } else if (pn < nu8) {
-              // each key block into its own accumulator, onto the bias the softmax left there
-              for (int t = 0; t < cnt; ++t) {
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-                  mma_i8_ta(tbase + (t ? TM_DB : TM_O), pt + 64 * t + 8 * kk,
-                            smem_desc(st + t * 64 * D + kk * 32, 16, 512, SW_64), idx8, 1u);
               }
             } else {
               const uint32_t pb = s0 + SM::P4 + (pn & 1) * SM::P4STRIDE;
@@ -546,13 +541,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto pfree_wait = [&](int v) -> bool {
       return v < 0 || mbar_wait(bar(B_P_FREE + (v & 1)), (uint32_t)(v >> 1) & 1u, spin);
     };
-    float ref = -INFINITY;    // O's reference per row: an integer, log2 units
+    float ref = -INFINITY;    // O's reference per row: an integer, log2 units (the shared statistics)
     float l = 0.f;            // this thread's part of the row sum, relative to 2^ref
     float x_run = -INFINITY;  // running row max (log2 units) over every unit so far
-    float O[DH];              // O in registers through the low-bit phases
     bool ok = true;
 #pragma unroll
     for (int c = 0; c < DH; c += 32) tmem_fill16x2_x32<DH>(tl + TM_O + c, 0u);  // O starts at zero
+    if (n4 > 0) {
+      tmem_fill16x2_x32<32>(tl + TM_L4, 0u);  // so do the 4-bit row sums
+      if (warp < 4) {
+        // warp w writes lane quarter w (32x32b shape): per 64-channel chunk the
+        // scale atoms of both query blocks (rows i, i+32 | i+64, i+96), and
+        // the ones tile's scales (all 1)
+        const uint32_t tq = tbase + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < H; ++c) {
+          uint32_t w[4];
+          const uint8_t* sa = A.q_sf4 + ((size_t)bh * g.nb + qa) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+          w[0] = *reinterpret_cast<const uint32_t*>(sa);
+          w[1] = *reinterpret_cast<const uint32_t*>(sa + 4);
+          if (qb >= 0) {
+            const uint8_t* sbp = A.q_sf4 + ((size_t)bh * g.nb + qb) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+            w[2] = *reinterpret_cast<const uint32_t*>(sbp);
+            w[3] = *reinterpret_cast<const uint32_t*>(sbp + 4);
+          } else {
+            w[2] = w[3] = 0u;
+          }
+          tmem_st4(tq + TM_SFQ + 4 * c, w);
+        }
+        const uint32_t one[4] = {kOneE4m3x4, kOneE4m3x4, kOneE4m3x4, kOneE4m3x4};
+        tmem_st4(tq + TM_SF1, one);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SFQ));
+      }
+    }
     tmem_wait_st();
     // item entries (and INT8 key scales) are loaded one unit ahead, so no unit
     // starts by waiting on global memory
@@ -571,6 +595,53 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int i0v, cntv;
       unit_items(u, i0v, cntv);
       return hh < cntv && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
+    };
+    // O (this thread's channels) times a per-row factor a and per-channel
+    // factors ch[] (ch == nullptr: none); the MMAs that write O have completed
+    auto scale_o = [&](float a, const float* ch) {
+#pragma unroll 1
+      for (int c = 0; c < DH; c += 32) {
+        uint32_t orr[32];
+        tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          orr[i] = __float_as_uint(__uint_as_float(orr[i]) * (ch ? a * ch[c + i] : a));
+        tmem_st16x2_x32<DH>(tl + TM_O + c, orr);
+      }
+      tmem_wait_st();
+    };
+    // the lazy reference of the 16-bit and INT8 phases: raised to ceil(um)
+    // only when the unit's row maximum um exceeds it by more than 2^8; returns
+    // the factor that O and l take (1 if unchanged)
+    auto lazy_raise = [&](float um, bool& need_o) -> float {
+      const bool need = um != -INFINITY && (ref == -INFINITY || um > ref + kRescaleThreshold);
+      need_o = need && ref != -INFINITY;
+      const float a = need_o ? pow2i(ref - ceilf(um)) : 1.0f;
+      if (need) ref = ceilf(um);
+      return a;
+    };
+    // a unit's P goes to TMEM in place of its scores; O, if its reference
+    // moved, is rescaled first (once the P·V of the unit before completed)
+    auto finish_unit = [&](int u, uint32_t sb, const uint32_t* pw, bool need_o, float a) -> bool {
+      if (__any_sync(FULL, need_o)) {
+        if (!__all_sync(FULL, pfree_wait(u - 1))) return false;
+        tc_fence_after();
+        scale_o(a, nullptr);
+      }
+      tmem_st16x2_x32<64>(sb, pw);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
+      return true;
+    };
+    // the last P·V before a phase boundary has completed (and O may be read)
+    auto boundary = [&](int last) -> bool {
+      if (last < 0) return true;
+      const bool done = __all_sync(FULL, pfree_wait(last));
+      tc_fence_after();
+      return done;
     };
 
     // ================================================================ 16-bit phase
@@ -604,10 +675,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       sk_next = sk_for(u + 1, e_next);
       const float um = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16)) * sl2;  // unit row max, log2 units
       x_run = fmaxf(x_run, um);
-      const bool need = um != -INFINITY && (ref == -INFINITY || um > ref + kRescaleThreshold);
-      const bool need_o = need && ref != -INFINITY;
-      const float a = need_o ? pow2i(ref - ceilf(um)) : 1.0f;
-      if (need) ref = ceilf(um);
+      bool need_o;
+      const float a = lazy_raise(um, need_o);
       uint32_t pw[32];
       if (member) {
         const uint64_t sl2x2 = f2pack(sl2, sl2), negm = f2pack(-ref, -ref);
@@ -630,99 +699,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int i = 0; i < 32; ++i) pw[i] = 0u;
         l *= a;
       }
-      // O can be rescaled once the P·V of unit u-1 completed; only then wait
-      if (__any_sync(FULL, need_o)) {
-        if (!__all_sync(FULL, pfree_wait(u - 1))) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t orr[32];
-          tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * a);
-          tmem_st16x2_x32<DH>(tl + TM_O + c, orr);
-        }
-      }
-      // P (bf16 pairs, key 2i in the low half of column i) replaces this
-      // thread's scores in TMEM, where the P·V MMA reads it
-      tmem_st16x2_x32<64>(sb, pw);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
+      if (!finish_unit(u, sb, pw, need_o, a)) { ok = false; break; }
     }
 
-    // ================================================================ low-bit phases
-    const bool lowbit = nu > nu16;
-    if (ok && lowbit) {
-      // O moves to registers; its TMEM columns become the low-bit accumulators
-      if (nu16 > 0) {
-        if (!__all_sync(FULL, pfree_wait(nu16 - 1))) ok = false;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t orr[32];
-          tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) O[c + i] = __uint_as_float(orr[i]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < DH; ++c) O[c] = 0.f;
-      }
-    }
-
-    // ---------------------------------------------------------------- INT8 phase
+    // ================================================================ INT8 phase
     if (ok && nu8 > nu16) {
-      // O in INT8 units (divided by the channel scale sv/255) while the phase runs
-      const float* inv8 = vsc + hh * DH;
-#pragma unroll
-      for (int c = 0; c < DH; ++c) O[c] *= inv8[c];
-      // D_a and D_b start from the bias
-#pragma unroll
-      for (int c = 0; c < DH; c += 32) {
-        tmem_fill16x2_x32<DH>(tl + TM_O + c, kI8Bias);
-        tmem_fill16x2_x32<DH>(tl + TM_DB + c, kI8Bias);
-      }
-      tmem_wait_st();
-      float x_own = -INFINITY, x_oth = -INFINITY;  // the last unit's block maxima of this row (log2)
-      uint32_t cs_own = 0;                         // the last unit's code sum of this thread's block
-      // fold the last unit's two accumulators into O with weights 2^(x_blk - ref)
-      auto fold8 = [&]() {
-        const float um = fmaxf(x_own, x_oth);
-        if (um != -INFINITY && (ref == -INFINITY || um > ref)) {
-          const float nr = ceilf(um);
-          const float a = ref == -INFINITY ? 0.f : pow2i(ref - nr);
-#pragma unroll
-          for (int c = 0; c < DH; ++c) O[c] *= a;
-          l *= a;
-          ref = nr;
-        }
-        const float w_own = x_own == -INFINITY ? 0.f : fast_exp2(x_own - ref);
-        const float w_oth = x_oth == -INFINITY ? 0.f : fast_exp2(x_oth - ref);
-        l = fmaf(w_own * (1.0f / 255.0f), (float)cs_own, l);
-        const float wa = hh == 0 ? w_own : w_oth, wb = hh == 0 ? w_oth : w_own;
-        const uint64_t wa2 = f2pack(wa, wa), wb2 = f2pack(wb, wb), nb2 = f2pack(-kI8BiasF, -kI8BiasF);
-#pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t da[32], db[32];
-          tmem_ld16x2_x32<DH>(tl + TM_O + c, da);
-          tmem_ld16x2_x32<DH>(tl + TM_DB + c, db);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            uint64_t o2 = f2pack(O[c + i], O[c + i + 1]);
-            o2 = f2fma(f2add(f2pack(__uint_as_float(da[i]), __uint_as_float(da[i + 1])), nb2), wa2, o2);
-            o2 = f2fma(f2add(f2pack(__uint_as_float(db[i]), __uint_as_float(db[i + 1])), nb2), wb2, o2);
-            f2unpack(o2, O[c + i], O[c + i + 1]);
-          }
-          tmem_fill16x2_x32<DH>(tl + TM_O + c, kI8Bias);
-          tmem_fill16x2_x32<DH>(tl + TM_DB + c, kI8Bias);
-        }
-        tmem_wait_st();
-      };
+      // O goes to INT8 units (divided by the V channel scale sv/255)
+      ok = boundary(nu16 - 1);
+      if (ok) scale_o(1.0f, vsc + VS_TO8 * D + hh * DH);
       for (int u = nu16; ok && u < nu8; ++u) {
         if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
         const uint32_t sb = tl + TM_S + (u & 1) * 128u;
@@ -755,137 +739,74 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           xh = (float)max(max(m4[0], m4[1]), max(m4[2], m4[3])) * sc;  // a member row has a real key
         }
         sk_next = sk_for(u + 1, e_next);
-        const float xo = __shfl_xor_sync(FULL, xh, 16);
-        x_run = fmaxf(x_run, fmaxf(xh, xo));
-        // codes round(255 p) with p = 2^(s*sc - x_blk) against the block's own maximum
-        uint32_t pw[16];
-        uint32_t csum = 0;
+        const float um = fmaxf(xh, __shfl_xor_sync(FULL, xh, 16));
+        x_run = fmaxf(x_run, um);
+        bool need_o;
+        const float a = lazy_raise(um, need_o);
+        uint32_t pw[32];
         if (member) {
-          const uint64_t scx2 = f2pack(sc, sc), negx = f2pack(-xh, -xh), kx2 = f2pack(-kI8BiasF, -kI8BiasF);
+          // codes c = round(255 p), p = 2^(s*sc - rb) against the block's own
+          // power-of-two reference rb; P = c * 2^(rb - ref), exact in bf16
+          const float rb = ceilf(xh);
+          const float s2k = pow2i(rb - ref);  // rb - ref <= 8
+          const uint64_t scx2 = f2pack(sc, sc), negr = f2pack(-rb, -rb), kx2 = f2pack(-kI8BiasF, -kI8BiasF);
           const uint64_t c255 = f2pack(255.0f, 255.0f), kmag = f2pack(kI8BiasF, kI8BiasF);
+          const uint64_t k2 = f2pack(s2k, s2k), nmk = f2pack(-kI8BiasF * s2k, -kI8BiasF * s2k);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            uint32_t c[4];
-#pragma unroll
-            for (int q = 0; q < 4; q += 2) {
-              const int k0 = 4 * i + q;
-              // the exact s32 -> fp32 conversion through the mantissa of 1.5*2^23 (|S| < 2^22)
-              const uint64_t sp = f2add(f2pack(__uint_as_float(sr[k0] + kI8Bias), __uint_as_float(sr[k0 + 1] + kI8Bias)), kx2);
-              float x0, x1;
-              f2unpack(f2fma(sp, scx2, negx), x0, x1);
-              float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              if (!full) {  // padding keys contribute nothing, whatever the block scale (sc may be 0)
-                if (!((vm >> k0) & 1ull)) p0 = 0.f;
-                if (!((vm >> (k0 + 1)) & 1ull)) p1 = 0.f;
-              }
-              float r0, r1;  // 255 p + 1.5*2^23: round-to-nearest-even code in the low byte
-              f2unpack(f2fma(f2pack(p0, p1), c255, kmag), r0, r1);
-              c[q] = __float_as_uint(r0);
-              c[q + 1] = __float_as_uint(r1);
+          for (int i = 0; i < 32; ++i) {
+            const int k0 = 2 * i;
+            // the exact s32 -> fp32 conversion through the mantissa of 1.5*2^23 (|S| < 2^22)
+            const uint64_t sp = f2add(f2pack(__uint_as_float(sr[k0] + kI8Bias), __uint_as_float(sr[k0 + 1] + kI8Bias)), kx2);
+            float x0, x1;
+            f2unpack(f2fma(sp, scx2, negr), x0, x1);
+            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            if (!full) {  // padding keys contribute nothing, whatever the block scale (sc may be 0)
+              if (!((vm >> k0) & 1ull)) p0 = 0.f;
+              if (!((vm >> (k0 + 1)) & 1ull)) p1 = 0.f;
             }
-            pw[i] = pack_low_bytes(c[0], c[1], c[2], c[3]);
-            csum = __dp4a(pw[i], 0x01010101u, csum);
+            // 255 p + 1.5*2^23 holds the round-to-nearest-even code; times 2^k minus 1.5*2^23*2^k is c*2^k exactly
+            const uint64_t w2 = f2fma(f2fma(f2pack(p0, p1), c255, kmag), k2, nmk);
+            acc[i & 3] = f2add(acc[i & 3], w2);
+            float w0, w1;
+            f2unpack(w2, w0, w1);
+            pw[i] = __byte_perm(__float_as_uint(w0), __float_as_uint(w1), 0x7632);  // the two bf16 halves
           }
+          float s0_, s1_, s2_, s3_;
+          f2unpack(f2add(acc[0], acc[1]), s0_, s1_);
+          f2unpack(f2add(acc[2], acc[3]), s2_, s3_);
+          l = l * a + ((s0_ + s1_) + (s2_ + s3_)) * (1.0f / 255.0f);
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pw[i] = 0u;
+          for (int i = 0; i < 32; ++i) pw[i] = 0u;
+          l *= a;
         }
-        // the codes (four per column, key 4i in the low byte) replace this
-        // thread's scores in TMEM, where the P·V MMA reads them
-        tmem_st16x2_x16<64>(sb, pw);
-        tmem_wait_st();
-        // the unit before: its accumulators are read once its P·V completed,
-        // and must be before this unit's P·V writes them
-        if (u > nu16) {
-          if (!__all_sync(FULL, pfree_wait(u - 1))) { ok = false; break; }
-          tc_fence_after();
-          fold8();
-        }
-        x_own = xh; x_oth = xo; cs_own = csum;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
-      }
-      if (ok) {
-        if (!__all_sync(FULL, pfree_wait(nu8 - 1))) ok = false;
-        tc_fence_after();
-        if (ok) fold8();
+        if (!finish_unit(u, sb, pw, need_o, a)) { ok = false; break; }
       }
       // back to value units
-      const float* fwd8 = vsc + D + hh * DH;
-#pragma unroll
-      for (int c = 0; c < DH; ++c) O[c] *= fwd8[c];
+      if (ok) ok = boundary(nu8 - 1);
+      if (ok) scale_o(1.0f, vsc + VS_FROM8 * D + hh * DH);
     }
 
-    // ---------------------------------------------------------------- 4-bit phase
+    // ================================================================ 4-bit phase
     if (ok && nu > nu8) {
-      const float* g4 = vsc + 2 * D + hh * DH;  // g/2688 of this thread's channels
-      // the 4-bit TMEM area: O4 and L4 at zero, Q's and the ones tile's scale factors
-#pragma unroll
-      for (int c = 0; c < DH; c += 32) tmem_fill16x2_x32<DH>(tl + TM_O + c, 0u);
-      tmem_fill16x2_x32<32>(tl + TM_L4, 0u);
-      if (warp < 4) {
-        // warp w writes lane quarter w (32x32b shape): per 64-channel chunk the
-        // scale atoms of both query blocks (rows i, i+32 | i+64, i+96)
-        const uint32_t tq = tbase + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-        for (int c = 0; c < H; ++c) {
-          uint32_t w[4];
-          const uint8_t* sa = A.q_sf4 + ((size_t)bh * g.nb + qa) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
-          w[0] = *reinterpret_cast<const uint32_t*>(sa);
-          w[1] = *reinterpret_cast<const uint32_t*>(sa + 4);
-          if (qb >= 0) {
-            const uint8_t* sbp = A.q_sf4 + ((size_t)bh * g.nb + qb) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
-            w[2] = *reinterpret_cast<const uint32_t*>(sbp);
-            w[3] = *reinterpret_cast<const uint32_t*>(sbp + 4);
-          } else {
-            w[2] = w[3] = 0u;
-          }
-          tmem_st4(tq + TM_SFQ + 4 * c, w);
-        }
-        const uint32_t one[4] = {kOneE4m3x4, kOneE4m3x4, kOneE4m3x4, kOneE4m3x4};
-        tmem_st4(tq + TM_SF1, one);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_F4));
-      // one power-of-two reference per row for the whole phase, from the
-      // running maximum of the earlier phases (the shared statistics)
-      float r4 = x_run == -INFINITY ? -INFINITY : ceilf(x_run);
-      // O4 and L4 join O (rows in `sel`) with weight 2^(r4 - ref) and restart at zero
-      auto fold4 = [&](bool sel) {
-        float w = 0.f;
-        if (sel && r4 != -INFINITY) {
-          if (ref == -INFINITY || r4 > ref) {
-            const float a = ref == -INFINITY ? 0.f : pow2i(ref - r4);
-#pragma unroll
-            for (int c = 0; c < DH; ++c) O[c] *= a;
-            l *= a;
-            ref = r4;
-          }
-          w = pow2i(r4 - ref);
-        }
+      // O goes to 4-bit units (divided by g/2688), against a reference raised
+      // to the ceiling of the running maximum, so that the phase's P stays in
+      // (0, 1] and later raises are rare
+      ok = boundary(nu8 - 1);
+      const float r0 = x_run == -INFINITY ? ref : (ref == -INFINITY ? ceilf(x_run) : fmaxf(ref, ceilf(x_run)));
+      const float a0 = (ref == -INFINITY || r0 == ref) ? 1.0f : pow2i(ref - r0);
+      ref = r0;
+      l *= a0;
+      if (ok) scale_o(a0, vsc + VS_TO4 * D + hh * DH);
+      // L4 (the quantised row sums, relative to 2^ref) joins l; rows in `sel` only
+      auto fold_l4 = [&](bool sel, float a) {
         uint32_t lv;
         tmem_ld16x2_x1<32>(tl + TM_L4, lv);
         tmem_wait_ld();
-        if (sel && hh == 0) l = fmaf(w * (1.0f / kP4Range), __uint_as_float(lv), l);
-#pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t o4[32];
-          tmem_ld16x2_x32<DH>(tl + TM_O + c, o4);
-          tmem_wait_ld();
-          if (sel) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              O[c + i] = fmaf(__uint_as_float(o4[i]), w * g4[c + i], O[c + i]);
-              o4[i] = 0u;
-            }
-          }
-          tmem_st16x2_x32<DH>(tl + TM_O + c, o4);
-        }
+        if (sel && hh == 0) l = fmaf(__uint_as_float(lv), 1.0f / kP4Range, l);
+        if (sel) l *= a;
         tmem_fill16x2_x32<32>(tl + TM_L4, sel ? 0u : lv);
-        tmem_wait_st();
       };
       for (int u = nu8; ok && u < nu; ++u) {
         if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
@@ -919,22 +840,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;
         }
         const float um = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));  // the unit's row maximum
-        // the reference rises to ceil(max) whenever the max exceeds it: what
-        // the phase holds joins O first, once the P·V of the unit before completed
-        const bool raise = um != -INFINITY && (r4 == -INFINITY || um > r4);
-        const bool held = raise && r4 != -INFINITY;  // rows with something accumulated to fold first
-        if (__any_sync(FULL, held)) {
+        // the reference rises to ceil(max) whenever the max exceeds it: O and
+        // the row sums are rescaled first, once the P·V of the unit before completed
+        const bool raise = um != -INFINITY && (ref == -INFINITY || um > ref);
+        const float a = (raise && ref != -INFINITY) ? pow2i(ref - ceilf(um)) : 1.0f;
+        if (__any_sync(FULL, raise)) {
           if (!__all_sync(FULL, pfree_wait(u - 1))) { ok = false; break; }
           tc_fence_after();
-          fold4(held);
+          fold_l4(raise, a);
+          scale_o(a, nullptr);
         }
-        if (raise) r4 = ceilf(um);
+        if (raise) ref = ceilf(um);
         uint32_t pw[8];
         uint32_t sfw = 0u;  // the row's four e4m3 P scales
 #pragma unroll
         for (int i = 0; i < 8; ++i) pw[i] = 0u;
         if (member) {
-          const uint64_t sl2x2 = f2pack(sl2, sl2), negr = f2pack(-r4, -r4);
+          const uint64_t sl2x2 = f2pack(sl2, sl2), negr = f2pack(-ref, -ref);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             float x0, x1;
@@ -983,19 +905,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
       }
-      // the phase joins O once its last P·V completed
+      // the phase's row sums join l and O returns to value units
+      if (ok) ok = boundary(nu - 1);
       if (ok) {
-        if (!__all_sync(FULL, pfree_wait(nu - 1))) ok = false;
-        tc_fence_after();
-        if (ok) fold4(true);
+        fold_l4(true, 1.0f);
+        scale_o(1.0f, vsc + VS_FROM4 * D + hh * DH);
       }
     }
     if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
     // ---- epilogue: O / l in bf16, staged for the TMA store
     {
-      if (ok && !lowbit && nu16 > 0) {
-        if (!__all_sync(FULL, pfree_wait(nu16 - 1))) { raise_timeout(A.status); *abort_flag = 1; }
-        tc_fence_after();
+      if (ok && nu16 == nu && nu > 0) {
+        // only the 16-bit phase ran: its last P·V completes before O is read
+        if (!boundary(nu - 1)) { raise_timeout(A.status); *abort_flag = 1; }
       }
       const float lt = l + __shfl_xor_sync(FULL, l, 16);
       const float il = lt > 0.f ? 1.0f / lt : 0.f;
@@ -1004,23 +926,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int chunk0 = D == 128 ? 0 : 4 * hh;  // 16-byte chunk of this thread's first channel
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
-        float v[32];
-        if (lowbit) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = O[c + i];
-        } else {
-          uint32_t orr[32];
-          tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(orr[i]);
-        }
+        uint32_t orr[32];
+        tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
+        tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t w[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 hb = __floats2bfloat162_rn(v[8 * q + 2 * i] * il, v[8 * q + 2 * i + 1] * il);
+            __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(orr[8 * q + 2 * i]) * il,
+                                                      __uint_as_float(orr[8 * q + 2 * i + 1]) * il);
             w[i] = *reinterpret_cast<uint32_t*>(&hb);
           }
           const int chunk = chunk0 + (c >> 3) + q;
@@ -1146,6 +1061,17 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t rowbytes
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 matrix [rows][cols] in boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t cols, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Status word of the dense path (its waits are bounded like the sparse
 // path's; the dense entry point has no workspace to report through).
 __device__ int g_dense_status;
@@ -1208,7 +1134,7 @@ cudaError_t launch_attention_tc(const Geom& g, const Layout& L, const void* q, c
       !make_region_map(&m[2], v, g, true) || !make_region_map(&m[3], out, g, true) ||
       !map_rows(&m[4], at<int8_t>(ws, L, R_Q_I8), rows64, D, 64, sw8) ||
       !map_rows(&m[5], at<int8_t>(ws, L, R_K_I8), rows64, D, 64, sw8) ||
-      !map_rows(&m[6], at<int8_t>(ws, L, R_V_I8), rowsD, 64, D, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map_bf16_rows(&m[6], at<__nv_bfloat16>(ws, L, R_V_I8), rows64, D, 64) ||
       !map_rows(&m[7], at<uint8_t>(ws, L, R_Q_F4), rows64, D / 2, 64, sw4) ||
       !map_rows(&m[8], at<uint8_t>(ws, L, R_K_F4), rows64, D / 2, 64, sw4) ||
       !map_rows(&m[9], at<uint8_t>(ws, L, R_V_F4), rowsD, 32, D, CU_TENSOR_MAP_SWIZZLE_32B))

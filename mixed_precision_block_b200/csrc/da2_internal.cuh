@@ -75,7 +75,7 @@ inline Layout make_layout(const Geom& g) {
   L.size[R_Q_S8] = L.size[R_K_S8] = bh * nb * 4;
   L.size[R_Q_F4] = L.size[R_K_F4] = bh * nb * S * d / 2;
   L.size[R_Q_SF4] = L.size[R_K_SF4] = bh * nb * (d / 64) * kSfAtomBytes;
-  L.size[R_V_I8] = bh * nb * d * S;
+  L.size[R_V_I8] = bh * nb * S * d * 2;  // INT8 codes held as bf16 values, [slot][channel] per block
   L.size[R_V_S8] = bh * d * 4;
   L.size[R_V_F4] = bh * nb * d * S / 2;
   L.size[R_V_SF4] = bh * nb * kSfAtomBytes;

@@ -44,17 +44,6 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   }
 }
 
-__device__ __forceinline__ uint32_t quant_i8x4(const float* x, float inv) {
-  uint32_t r = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int c = __float2int_rn(__fmul_rn(x[i], inv));
-    c = max(-127, min(127, c));
-    r |= (uint32_t)(c & 0xff) << (8 * i);
-  }
-  return r;
-}
-
 // NVFP4 microblock of 16 values held as 8 per lane in lanes (2j, 2j+1):
 // returns 4 code bytes for this lane's 8 values and the e4m3 scale byte.
 __device__ __forceinline__ uint32_t quant_f4x8(const float* x, float amax16, uint32_t* sf_byte) {
@@ -298,7 +287,7 @@ __global__ void __launch_bounds__(kThreads) v_amax_kernel(Geom g, const __nv_bfl
 struct VPtrs {
   const __nv_bfloat16* v;
   const unsigned int* amax_bits;
-  int8_t* i8;
+  __nv_bfloat16* q8;  // INT8 codes as bf16 values, [block][slot][channel]
   float* s8;
   uint8_t* f4;
   uint8_t* sf4;
@@ -378,20 +367,27 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
       if (want_f4) P.g4[(size_t)bh * D + tid] = __fdiv_rn(a, 2688.0f);
     }
     if (!active) continue;
+    if (want_i8) {
+      // the codes of channels c0, c0+1 for this thread's 16 slots, as bf16
+      // values (integers up to 127: exact), in the block's [slot][channel]
+      // order — the layout of a bf16 V tile, so the INT8 phase's P·V runs on
+      // the same tensor-core path as the 16-bit phase's
+      const float a0 = __uint_as_float(amax_bits[c0]), a1 = __uint_as_float(amax_bits[c0 + 1]);
+      const float inv0 = a0 > 0.f ? __fdiv_rn(127.0f, a0) : 0.f, inv1 = a1 > 0.f ? __fdiv_rn(127.0f, a1) : 0.f;
+      __nv_bfloat16* dst = P.q8 + (blk_lin * 64 + 16 * j) * D + c0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int k0 = max(-127, min(127, __float2int_rn(__fmul_rn(f0[e], inv0))));
+        const int k1 = max(-127, min(127, __float2int_rn(__fmul_rn(f1[e], inv1))));
+        *reinterpret_cast<__nv_bfloat162*>(dst + (size_t)e * D) =
+            __floats2bfloat162_rn((float)k0, (float)k1);
+      }
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float* f = h ? f1 : f0;
       const int c = c0 + h;
       const float a = __uint_as_float(amax_bits[c]);
-      if (want_i8) {
-        const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
-        uint4 w;
-        w.x = quant_i8x4(f, inv);
-        w.y = quant_i8x4(f + 4, inv);
-        w.z = quant_i8x4(f + 8, inv);
-        w.w = quant_i8x4(f + 12, inv);
-        *reinterpret_cast<uint4*>(P.i8 + (blk_lin * D + c) * 64 + 16 * j) = w;
-      }
       if (want_f4) {
         const float gch = __fdiv_rn(a, 2688.0f);
         const float r = gch > 0.f ? __fdiv_rn(1.0f, gch) : 0.f;
@@ -450,7 +446,7 @@ cudaError_t launch_prepare_d(const Geom& g, const Layout& L, const void* q, cons
   v_amax_kernel<D><<<dim3((g.N + tpc - 1) / tpc, g.BH), kThreads, 0, st>>>(
       g, static_cast<const __nv_bfloat16*>(v), amax, tpc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  VPtrs V{static_cast<const __nv_bfloat16*>(v), amax, at<int8_t>(ws, L, R_V_I8),
+  VPtrs V{static_cast<const __nv_bfloat16*>(v), amax, at<__nv_bfloat16>(ws, L, R_V_I8),
           at<float>(ws, L, R_V_S8), at<uint8_t>(ws, L, R_V_F4), at<uint8_t>(ws, L, R_V_SF4),
           at<float>(ws, L, R_V_G4)};
   CUtensorMap tv;

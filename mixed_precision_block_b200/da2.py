@@ -222,7 +222,7 @@ def view(p, ws, which) -> torch.Tensor:
         "Q_S8": (torch.float32, (BH, nb)), "K_S8": (torch.float32, (BH, nb)),
         "Q_F4": (torch.uint8, (BH, nb, 64, d // 2)), "K_F4": (torch.uint8, (BH, nb, 64, d // 2)),
         "Q_SF4": (torch.uint8, (BH, nb, d // 64, 32, 16)), "K_SF4": (torch.uint8, (BH, nb, d // 64, 32, 16)),
-        "V_I8": (torch.int8, (BH, nb, d, 64)), "V_S8": (torch.float32, (BH, d)),
+        "V_I8": (torch.bfloat16, (BH, nb, 64, d)), "V_S8": (torch.float32, (BH, d)),
         "V_F4": (torch.uint8, (BH, nb, d, 32)), "V_SF4": (torch.uint8, (BH, nb, 32, 16)),
         "V_G4": (torch.float32, (BH, d)),
         "SCORES": (torch.float32, (BH, nb, nb)), "MAP": (torch.uint8, (BH, nb, nb)),

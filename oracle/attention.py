@@ -22,20 +22,22 @@ Readings adopted (the pages leave these open):
   integer product of the INT8 codes times both block scales; 4-bit phase from
   the dequantised NVFP4 values; all times 1/sqrt(d).  Padding keys score -inf.
 * low-bit P is quantised per (query row, key block), relative to that block's
-  own row maximum, so that every retained block keeps the full resolution of
-  its format whatever its rank in the row (the reading note, Method overview
-  bullet 3: low-bit precision recovers the mid-importance interactions):
-  - 8-bit: p = exp(s - m_blk) in (0, 1], m_blk the block's row maximum;
-    code = round(255 p) as an unsigned byte; the block's weights are code/255
-    times exp(m_blk - m);
-  - 4-bit: with x = s log2 e, the reference is r_blk = ceil(max x), the
-    block's row maximum rounded up to a power of two; p = 2^(x - r_blk) in
-    (0, 1] is quantised as NVFP4 of 2688 p over 16 consecutive keys of the
-    row (2688 = 6 x 448 puts the largest possible p at the top of the
-    e2m1 x e4m3 range), dequantised and divided by 2688; the block's weights
-    are that times 2^r_blk.  A power of two passes through the e4m3 scale
-    exactly, so the same codes come out against any larger power-of-two
-    reference while the microblock scale stays normal (>= 2^-6).
+  own row maximum rounded up to a power of two: with x = s log2 e, the
+  reference is r_blk = ceil(max x) and p = 2^(x - r_blk) in (0, 1].  Every
+  retained block so keeps the full resolution of its format whatever its rank
+  in the row (the reading note, Method overview bullet 3: low-bit precision
+  recovers the mid-importance interactions), and since its scale 2^r_blk is a
+  power of two, its weights enter the shared accumulator exactly, with no
+  separate merge per block (bullet 4: the phases rescale at their boundaries
+  and avoid repeated write-backs and merges):
+  - 8-bit: code = round(255 p) as an unsigned byte; weights code/255 times
+    2^r_blk;
+  - 4-bit: NVFP4 of 2688 p over 16 consecutive keys of the row (2688 = 6 x 448
+    puts the largest possible p at the top of the e2m1 x e4m3 range),
+    dequantised and divided by 2688; weights that times 2^r_blk.  A power of
+    two passes through the e4m3 scale exactly, so the same codes come out
+    against any larger power-of-two reference while the microblock scale
+    stays normal (>= 2^-6).
 * the softmax denominator sums, per phase, the weights the numerator uses:
   unquantised p in the 16-bit phase, the quantised weights above in the
   low-bit phases (so each low-bit block enters numerator and denominator with
@@ -99,24 +101,30 @@ def _exp_rel(s, m):
     return np.where(ok, np.exp(np.where(ok, s - np.where(np.isfinite(m), m, 0)[:, None], 0)), 0.0)
 
 
-def p8_weights(s):
-    """8-bit phase weights of one key block (rows x keys, natural-log scores,
-    -inf for keys the row does not use): returns (m_blk, w) with
-    w = round(255 exp(s - m_blk)) / 255 relative to exp(m_blk)."""
-    m_blk = _row_max(s)
-    p = _exp_rel(s, m_blk)
-    return m_blk, np.rint(255.0 * p) / 255.0
+def _pow2_reference(x):
+    """Per row: r = ceil(max x) (-inf for a row without a finite score) and
+    p = 2^(x - r), 0 where x is -inf."""
+    xm = _row_max(x)
+    live = np.isfinite(xm)
+    r_blk = np.where(live, np.ceil(np.where(live, xm, 0.0)), -np.inf)
+    ok = np.isfinite(x) & live[:, None]
+    p = np.where(ok, np.exp2(np.where(ok, x - np.where(live, r_blk, 0.0)[:, None], 0.0)), 0.0)
+    return r_blk, p
+
+
+def p8_weights(x):
+    """8-bit phase weights of one key block (rows x keys, log2-unit scores,
+    -inf for unused keys): returns (r_blk, w) with r_blk = ceil(row max) and
+    w = round(255 * 2^(x - r_blk)) / 255 relative to 2^r_blk."""
+    r_blk, p = _pow2_reference(x)
+    return r_blk, np.rint(255.0 * p) / 255.0
 
 
 def p4_weights(x):
     """4-bit phase weights of one key block (rows x keys, log2-unit scores,
     -inf for unused keys): returns (r_blk, w) with r_blk = ceil(row max) and
     w = NVFP4(2688 * 2^(x - r_blk)) / 2688 relative to 2^r_blk."""
-    xm = _row_max(x)
-    live = np.isfinite(xm)
-    r_blk = np.where(live, np.ceil(np.where(live, xm, 0.0)), -np.inf)
-    ok = np.isfinite(x) & live[:, None]
-    p = np.where(ok, np.exp2(np.where(ok, x - np.where(live, r_blk, 0.0)[:, None], 0.0)), 0.0)
+    r_blk, p = _pow2_reference(x)
     t = F.f32(P4_RANGE * F.f32(p))
     codes, sf = F.nvfp4_quantize(t, axis=-1, block=16)
     return r_blk, F.nvfp4_dequantize(codes, sf) / P4_RANGE
@@ -150,7 +158,7 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
         st.merge(m_blk, p.sum(1), p_num @ prep["v_blocks"][kb])
 
     # phase 8: INT8 Q/K codes with block scales; u8 P against each block's own
-    # row maximum; INT8 V codes; the V channel scale applied at the boundary
+    # power-of-two reference; INT8 V codes; the V channel scale applied at the boundary
     kbs = np.nonzero(prec_row == BIT8)[0]
     if len(kbs):
         qi = prep["q_i8"][qb].astype(np.float64)
@@ -158,9 +166,9 @@ def qblock_attention(prep, qb, prec_row, d, mode="emulate"):
         ph = _State(S, d)
         for kb in kbs:
             s_int = qi @ prep["k_i8"][kb].astype(np.float64).T  # exact integers
-            s = np.where(valid[kb][None, :], s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d), -np.inf)
-            m_blk, w = p8_weights(s)
-            ph.merge(m_blk, w.sum(1), w @ prep["v_i8"][kb].astype(np.float64).T)
+            x = np.where(valid[kb][None, :], s_int * (sq * prep["k_s8"][kb] * inv_sqrt_d * LOG2E), -np.inf)
+            r_blk, w = p8_weights(x)
+            ph.merge(r_blk * LN2, w.sum(1), w @ prep["v_i8"][kb].astype(np.float64).T)
         st.merge(ph.m, ph.l, ph.o * prep["v_s8"][None, :])
 
     # phase 4: NVFP4 Q/K, NVFP4 P (16-key microblocks of 2688 p against each

@@ -106,7 +106,9 @@ def check_prep_head(p, ws, op, pr, bh, n8, n4, blocks=None):
             np.testing.assert_array_equal(qk_sf_natural(g(p, ws, f"{T}_SF4", bh))[sel], pr[f"{t}_sf4"][sel],
                                           err_msg=f"{T}_SF4")
     if n8:
-        np.testing.assert_array_equal(g(p, ws, "V_I8", bh)[sel], pr["v_i8"][sel], err_msg="V_I8")
+        # V's INT8 codes are held as bf16 values in [block][slot][channel] order
+        v8 = da2.view(p, ws, "V_I8")[bh].float().cpu().numpy().astype(np.int64).transpose(0, 2, 1)
+        np.testing.assert_array_equal(v8[sel], pr["v_i8"][sel].astype(np.int64), err_msg="V_I8")
         np.testing.assert_array_equal(g(p, ws, "V_S8", bh).astype(np.float64), pr["v_s8"])
     if n4:
         np.testing.assert_array_equal(unpack_nibbles(da2.view(p, ws, "V_F4")[bh])[sel], pr["v_f4"][sel],

@@ -21,8 +21,8 @@ denominator summing the quantised weights the numerator uses.
 
     python tests/readings_report.py [--qblocks 48]
 
-The adopted reading (oracle/attention.py) is INT8 blk_exact + ql and NVFP4
-blk_pow2 + ql.
+The adopted reading (oracle/attention.py) is blk_pow2 + ql for both low-bit
+formats.
 """
 
 from __future__ import annotations

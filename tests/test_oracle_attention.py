@@ -117,19 +117,24 @@ def _dequant_dense(p, pr, fmt):
 
 
 def test_p8_weights_by_hand():
-    # one row, keys with scores 0, ln(1/2), ln(1/4), -10 and an unused key:
-    # p = 1, 1/2, 1/4, e^-10 -> 255 p = 255, 127.5, 63.75, 0.0116 -> codes
-    # 255, 128 (the tie goes to the even code), 64, 0
-    s = np.array([[0.0, np.log(0.5), np.log(0.25), -10.0, -np.inf]])
-    m, w = attention.p8_weights(s)
-    assert m[0] == 0.0
-    np.testing.assert_array_equal(w * 255.0, [[255.0, 128.0, 64.0, 0.0, 0.0]])
-    # the reference is the block's own maximum: shifting every score keeps the
-    # codes (scores away from a rounding tie: 255 p = 255, 155.55 -> 156, 0)
-    s = np.array([[0.0, np.log(0.61), -10.0]])
-    m2, w2 = attention.p8_weights(s - 37.25)
-    assert m2[0] == -37.25
-    np.testing.assert_array_equal(w2 * 255.0, [[255.0, 156.0, 0.0]])
+    # one row, keys with log2 scores 0.3, -0.7, -1.7, -13 and an unused key:
+    # r = ceil(0.3) = 1; p = 2^-0.7 = 0.61557, 2^-1.7 = 0.30779, 2^-2.7 =
+    # 0.15389, 2^-14; 255 p = 156.97, 78.49, 39.24, 0.0156 -> codes 157, 78,
+    # 39, 0
+    x = np.array([[0.3, -0.7, -1.7, -13.0, -np.inf]])
+    r, w = attention.p8_weights(x)
+    assert r[0] == 1.0
+    np.testing.assert_array_equal(w * 255.0, [[157.0, 78.0, 39.0, 0.0, 0.0]])
+    # a block max on an integer: p = 1 exactly, code 255; midpoints go to the
+    # even code (255 * 2^-1 = 127.5 -> 128)
+    r, w = attention.p8_weights(np.array([[2.0, 1.0]]))
+    assert r[0] == 2.0
+    np.testing.assert_array_equal(w * 255.0, [[255.0, 128.0]])
+    # the reference is the block's own: shifting every score by an integer
+    # keeps the codes
+    r2, w2 = attention.p8_weights(x - 37.0)
+    assert r2[0] == -36.0
+    np.testing.assert_array_equal(w2, attention.p8_weights(x)[1])
 
 
 def test_p4_weights_by_hand():
@@ -185,10 +190,10 @@ def _two_level_head(d=64):
 @pytest.mark.parametrize("fmt", [8, 4])
 def test_low_bit_block_far_below_keeps_its_own_reference(fmt):
     # block 0 at 16 bits scores 8, block 1 in the low-bit phase scores 0: its
-    # p is taken against its own maximum (p = 1: INT8 code 255; NVFP4 2688 p =
-    # 2688 exactly), so its 64 keys enter numerator and denominator with
-    # weight e^-8 each.  (Against a shared running maximum the INT8 codes would
-    # be round(255 e^-8) = 0.)
+    # p is taken against its own reference 2^ceil(0) = 1 (p = 1: INT8 code 255;
+    # NVFP4 2688 p = 2688 exactly), so its 64 keys enter numerator and
+    # denominator with weight e^-8 each.  (Against a shared running maximum
+    # the INT8 codes would be round(255 e^-8) = 0.)
     p, pr, v, tab = _two_level_head()
     row = np.array([16, fmt, 0], dtype=np.uint8)
     out = attention.qblock_attention(pr, 0, row, p.d, "math")
@@ -218,8 +223,8 @@ def _alternating_head(d=64):
 @pytest.mark.parametrize("fmt", [8, 4])
 def test_low_bit_weights_enter_the_denominator_quantised(fmt):
     # INT8: q codes 127 (scale 8/127), k codes 0 and -127 (scale 0.75/127):
-    # scores 0 and -0.75; p = 1 and e^-0.75 = 0.47237; codes 255 and
-    # round(120.45) = 120.  NVFP4: q = 8 -> scale e4m3(8/6) = 1.375, code 6,
+    # scores 0 and -0.75, x = 0 and -1.082 log2, reference 2^0; p = 1 and
+    # 2^-1.082 = 0.47237; codes 255 and round(120.45) = 120.  NVFP4: q = 8 -> scale e4m3(8/6) = 1.375, code 6,
     # so 8.25; k = -0.75 exactly; scores 0 and -0.7734, x = 0 and -1.1158 log2;
     # p = 1 and 0.4614; one 16-key microblock holds both, scale e4m3(2688/6) =
     # 448, codes 6 and e2m1(1240.3/448 = 2.77) = 3: weights 1 and 1/2.  The
@@ -265,10 +270,10 @@ def test_low_bit_phase_within_p_quantisation_bound(fmt):
     exact = _sdpa(qd, kd, vd)
     # The output is sum(w~ v) / sum(w~) with w~ the quantised weights; against
     # the exact weights w: out - exact = sum((w~ - w)(v - exact)) / sum(w~).
-    # Each |w~ - w| <= e exp(m_blk - m), e the largest rounding error of one
-    # quantised p relative to its block reference (INT8: half a step of
-    # 1/255; NVFP4 against a power of two up to 2x above the block max: the
-    # top e2m1 half-step of the scale plus the scale's own rounding, < 0.18).
+    # Each |w~ - w| <= e 2^r_blk, e the largest rounding error of one
+    # quantised p relative to its block's power-of-two reference (INT8: half a
+    # step of 1/255; NVFP4: the top e2m1 half-step of the scale plus the
+    # scale's own rounding, < 0.18).
     e = 0.5 / 255 if fmt == 8 else 0.18
     s = qd @ kd.T / np.sqrt(p.d)
     tab = r["prep"]["table"]
@@ -278,8 +283,7 @@ def test_low_bit_phase_within_p_quantisation_bound(fmt):
     for b in range(p.nb):
         toks = tab[b][tab[b] >= 0]
         mb[:, toks] = s[:, toks].max(1, keepdims=True)
-    if fmt == 4:
-        mb = np.ceil(mb * attention.LOG2E) * attention.LN2  # the power-of-two reference
+    mb = np.ceil(mb * attention.LOG2E) * attention.LN2  # the power-of-two reference
     dw = e * np.exp(mb - m[:, None])
     w_low = np.maximum(w.sum(1) - dw.sum(1), 1e-300)
     bound = (np.einsum("nk,nkd->nd", dw, np.abs(vd[None, :, :] - exact[:, None, :]))) / w_low[:, None]
