@@ -159,6 +159,15 @@ int da2_attention_wait_test(const da2_problem* p, const void* q, const void* k, 
                             void* ws, size_t ws_bytes, void* out, int withheld_cta,
                             unsigned int wait_polls, void* stream);
 
+/* Introspection, no counterpart on the pages: *ctas_per_sm receives how many
+ * CTAs of the attention kernel for head dimension d (64 or 128; dense != 0:
+ * the dense kernel) one SM holds at once.  The kernel is laid out for 1 CTA
+ * per SM (it allocates all 512 TMEM columns, 384 threads at 168 registers)
+ * holding two query-block pairs, whose softmax warpgroups hide each other's
+ * latency.  Sets the kernel's launch attributes as a call would; no device
+ * work.  DA2_ERR_ARG for another d or a null pointer. */
+int da2_attention_occupancy(int d, int dense, int* ctas_per_sm);
+
 /* Workspace views for tests.  Returns the device address and size of one
  * intermediate inside `ws` (no device work).  Layouts (bh = b*H + h):
  *   PERM   int32 [nb][64]            token of each block slot, -1 = padding

@@ -220,6 +220,13 @@ int da2_attention_wait_test(const da2_problem* p, const void* q, const void* k, 
                                            withheld_cta));
 }
 
+int da2_attention_occupancy(int d, int dense, int* ctas_per_sm) {
+  if ((d != 64 && d != 128) || !ctas_per_sm) return DA2_ERR_ARG;
+  int rc = check_device();
+  if (rc) return rc;
+  return cuda_status(attention_occupancy(d, dense != 0, ctas_per_sm));
+}
+
 int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t* bytes) {
   Geom g;
   int rc = make_geom(p, &g);

@@ -12,49 +12,56 @@
 // tokens, so one query block gives an M = 64 MMA, which runs the tensor core at
 // half rate.  Each CTA owns a pair of neighbouring query blocks (2p, 2p+1) —
 // rows 0-63 and 64-127 of one M = 128 tile — and walks the merged key list of
-// the pair phase by phase, two key blocks (a "unit") at a time.  A key block
+// the pair phase by phase, one key block (a "unit") at a time.  A key block
 // only one of the two keeps is computed for all 128 rows and masked for the
-// other half.  Nothing a row computes depends on the other query block, nor on
-// the grouping into units, beyond rounding: every quantisation reference below
-// is the row's own per key block, and references are powers of two.
+// other half.  Nothing a row computes depends on the other query block beyond
+// rounding: every quantisation reference below is the row's own per key block,
+// and references are powers of two.
 //
-// Roles (12 warps).  Warps 0-7 do the softmax: warp w holds 16 tile rows,
-// 32(w&3) + 16(w>>2) + i, with two threads per row (lanes i and i+16), reading
-// TMEM with the 16x32bx2 shapes; lane i takes key block a of a unit (columns
-// 0-63 of its scores) and output channels [0, D/2), lane i+16 key block b and
-// channels [D/2, D).  The row maximum of a unit is one shuffle.  Warp 8 issues
-// TMA loads; warp 9 issues every MMA from a non-blocking scheduler; warps 10-11
-// only complete the third warpgroup, which hands most of its registers to the
-// softmax warpgroups.
+// Two tiles per CTA.  Tensor-memory kernels run one CTA per SM, so each CTA
+// holds two independent tile engines — two query-block pairs, each with its
+// own softmax warpgroup, TMA warp, MMA warp, 256 TMEM columns and shared-memory
+// half.  While one tile's softmax waits on a TMEM load, a barrier or its MMAs,
+// the other's exponentials keep the special-function unit busy, and the
+// tensor core alternates between the two tiles' score and P·V MMAs.
 //
-//   16-bit  S = Q·[K_a;K_b]^T (kind::f16, fp32 in TMEM, two buffers);
+// Roles (12 warps).  Warps 0-3 (tile 0) and 4-7 (tile 1) do the softmax, one
+// thread per tile row (TMEM lane), 64 scores per unit; warps 8 and 10 issue
+// the TMA loads of tiles 0 and 1, warps 9 and 11 their MMAs, each from a
+// non-blocking scheduler.
+//
+//   16-bit  S = Q·K^T (kind::f16, fp32 in TMEM, two buffers);
 //           P = exp2(s·log2e/√d − m) rounded to bf16 against an integer
 //           reference m per row (the shared statistics), raised lazily (O
 //           rescaled in TMEM only when the row max grows by more than 2^8); P
 //           replaces the scores in TMEM and O += P·V reads it from there (V
 //           MN-major from the TMA tile).
-//   8-bit   S8 = Q8·[K8_a;K8_b]^T (kind::i8, s32).  Per row and key block the
+//   8-bit   S8 = Q8·K8^T (kind::i8, s32).  Per row and key block the
 //           reference is the block's own maximum rounded up to a power of two,
 //           2^r_blk: codes c = round(255·2^(x − r_blk)).  c·2^(r_blk − m) is an
 //           8-bit integer times a power of two, exact in bf16, and so are the
 //           INT8 V codes: O += P·V8 runs on the 16-bit path (kind::f16, P from
 //           TMEM) straight into the shared accumulator, every product exact.
 //           The row sum takes the same weights /255.
-//   4-bit   S = Q4·K4_t^T (kind::mxf4nvf4, block16 ue4m3 scales copied into
+//   4-bit   S = Q4·K4^T (kind::mxf4nvf4, block16 ue4m3 scales copied into
 //           TMEM with tcgen05.cp); P = NVFP4 of 2688·2^(x − m) per 16 keys
 //           against the shared reference m, raised to the ceiling of the
 //           running maximum at the phase start and to a unit's maximum when
 //           it exceeds it (which reproduces each block's own power-of-two
 //           reference while the microscale stays normal); O += P4·V4 into the
-//           shared fp32 accumulator, and L4 += P4·1 (an MMA against a tile of
-//           e2m1 ones) gives the row sum of the quantised weights.
+//           shared fp32 accumulator.  The row sum of the quantised weights is
+//           exact integer arithmetic in the softmax thread: a byte permute
+//           maps four e2m1 codes to twice their values, a 4-way byte dot
+//           product adds them, one multiply applies the microscale.
 //   Around each low-bit phase O is multiplied by the inverse of the phase's V
 //   channel scale (sv/255 or g/2688) and back — the rescaling at the phase
 //   boundaries — so that the phase's MMAs work on the codes.
 // Operands arrive by TMA: bf16 Q/K/V as 8×8-token region boxes straight from
 // the [B,H,N,d] tensors (padding is the TMA zero fill), codes as 2-D boxes of
-// the workspace (V's INT8 codes held as bf16 values by the preparation).  The epilogue writes O / l through the same region box with a
-// TMA store, whose clipping drops the padding rows — the restore.
+// the workspace (V's INT8 codes held as bf16 values by the preparation).  Q8
+// and Q4 reuse Q's buffer once the last 16-bit score MMA has completed.  The
+// epilogue writes O / l through the same region box with a TMA store, whose
+// clipping drops the padding rows — the restore.
 // Every wait is bounded; on expiry the CTA raises its status word, stops
 // issuing, waits (bounded) for its own copies in flight and releases its
 // tensor memory.
@@ -72,14 +79,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kSoftmaxWarps = 8;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;  // warps 10-11 complete their warpgroup and idle
-constexpr int kThreads = 384;
-// Register split: launched at 168 per thread (three warps share a sub-partition's
-// 16K registers); the softmax warpgroups take 232, the producer/MMA warpgroup
-// 40: 2*128*232 + 128*40 = 384*168.
-constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 232, kRegsIssue = 40;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIssue <= kThreads * kRegsLaunch, "register split");
+constexpr int kTiles = 2;
+constexpr int kSoftmaxWarps = 4;  // per tile
+constexpr int kIssueWarp0 = 8;    // warps 8 + 2t (TMA) and 9 + 2t (MMA) serve tile t
+constexpr int kThreads = 384;  // 168 registers per thread: the SM's 64K registers
 constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -90,43 +93,42 @@ constexpr uint32_t kI8Bias = 0x4B400000u;
 constexpr float kI8BiasF = 12582912.0f;
 // the 4-bit phase quantises 2688 p: 6 (largest e2m1) x 448 (largest e4m3)
 constexpr float kP4Range = 2688.0f;
-constexpr uint32_t kOnesE2m1 = 0x22222222u;  // e2m1 1.0 in every nibble
-constexpr uint32_t kOneE4m3x4 = 0x38383838u; // ue4m3 1.0 in every byte
 constexpr uint32_t kDefaultSpin = 1u << 22;
 
-// TMEM columns (512 allocated).  [0, D): O, the one fp32 accumulator every
-// phase adds into.  [128, 384): two score buffers.  4-bit phase: scale factors
-// from 384 — Q 384, K_a 392, K_b 400, V_a 408, V_b 412, P_a 416, P_b 420,
-// ones 424 (all 4-aligned, as block-scaled MMAs require) — and the row sums of
-// the quantised P, L4, at 448 (64 columns).
-constexpr uint32_t TM_O = 0, TM_S = 128;
-constexpr uint32_t TM_SFQ = 384, TM_SFK = 392, TM_SFV = 408, TM_SFP = 416, TM_SF1 = 424, TM_L4 = 448;
+// TMEM columns (512 per CTA, 256 per tile, from the tile's base).  [0, D): O,
+// the one fp32 accumulator every phase adds into.  [128, 256): two score buffers of 64 columns (one key block).  The
+// 4-bit phase keeps its scores in the second buffer only (its P goes to shared
+// memory, so the buffer is free as soon as the softmax has read it) and its
+// scale factors over the first: Q 128, K 136/144 (two slots), V 152/156, P
+// 160/164 (all 4-aligned, as block-scaled MMAs require).
+constexpr uint32_t kTmemCols = 512, kTileCols = 256;
+constexpr uint32_t TM_O = 0, TM_S = 128, TM_S4 = 192;
+constexpr uint32_t TM_SFQ = 128, TM_SFK = 136, TM_SFV = 152, TM_SFP = 160;
 
-// Shared-memory map (offsets from a 1024-aligned base).
+// Shared-memory map: one half per tile (offsets from the tile's base, the
+// first 1024-aligned), then the CTA's MISC words.
 template <int D>
 struct Smem {
   static constexpr int H = D / 64;                         // 64-channel halves of a bf16 row
-  static constexpr uint32_t Q16 = 0;                       // [H][2 blocks][64 rows][128 B], SW128
-  static constexpr uint32_t Q8 = Q16 + 256u * D;           // [128 rows][D B]
-  static constexpr uint32_t Q4 = Q8 + 128u * D;            // [128 rows][D/2 B]
-  static constexpr uint32_t KR = Q4 + ((64u * D + 1023u) & ~1023u);  // K ring
-  static constexpr uint32_t STAGE = 256u * D;              // one ring slot: the largest unit (16-bit)
+  static constexpr uint32_t Q = 0;                         // Q16 [H][2 blocks][64 rows][128 B], SW128;
+                                                           // later Q8 [128 rows][D B] and Q4 at Q4OFF
+  static constexpr uint32_t Q4OFF = 128u * D;              // Q4 [128 rows][D/2 B]
+  static constexpr uint32_t KR = 256u * D;                 // K ring
+  static constexpr uint32_t STAGE = 128u * D;              // one ring slot: a bf16 key block
   static constexpr uint32_t VR = KR + kStages * STAGE;     // V ring
   static constexpr uint32_t P4 = VR + kStages * STAGE;     // two 4-bit P buffers
-  static constexpr uint32_t P4STRIDE = 10240;              // P4_a 4 KB | P4_b 4 KB | SF_a | SF_b
-  static constexpr uint32_t P4SF = 8192;
-  static constexpr uint32_t ONES = P4 + 2 * P4STRIDE;      // [64 rows][32 B] of e2m1 1.0
-  static constexpr uint32_t VS = ONES + 2048;              // fp32 [4][D] channel factors (see VS_*)
+  static constexpr uint32_t P4STRIDE = 5120;               // codes [128 rows][32 B] | scale atom
+  static constexpr uint32_t P4SF = 4096;
+  static constexpr uint32_t VS = P4 + 2 * P4STRIDE;        // fp32 [4][D] channel factors (see VS_*)
   static constexpr uint32_t BAR = VS + ((16u * D + 255u) & ~255u);
-  static constexpr uint32_t MISC = BAR + 512;
-  static constexpr uint32_t USED = MISC + 256;
-  // ask for at least 120 KB so that one CTA holds an SM (it allocates all of TMEM)
-  static constexpr uint32_t BYTES = (USED + 1024 > 120u * 1024) ? USED + 1024 : 120u * 1024;
-  // 4-bit units: K4_a | K4_b (or V4_a | V4_b) take 64·D bytes; scale atoms follow
-  static constexpr uint32_t SL_SF = 64u * D;
+  static constexpr uint32_t TILE = (BAR + 256u + 1023u) & ~1023u;
+  static constexpr uint32_t MISC = kTiles * TILE;          // TMEM base, abort flag, e4m3 reciprocals
+  static constexpr uint32_t BYTES = MISC + 256 + 1024;     // + alignment slack
+  // 4-bit slots: K4 (or V4) codes take 32·D bytes; scale atoms follow
+  static constexpr uint32_t SL_SF = 32u * D;
 };
 static_assert(Smem<128>::BYTES <= 227 * 1024, "shared memory");
-static_assert(Smem<64>::BYTES <= 227 * 1024, "shared memory");
+static_assert(Smem<128>::Q4OFF + 64u * 128 <= Smem<128>::KR, "Q8 and Q4 fit in Q's buffer");
 
 // channel factors that move O into a low-bit phase's units and back:
 // 255/sv, sv/255 (INT8: V codes times sv/255... P codes /255), 2688/g, g/2688
@@ -135,11 +137,11 @@ enum { VS_TO8 = 0, VS_FROM8 = 1, VS_TO4 = 2, VS_FROM4 = 3 };
 
 // mbarrier slots (8 bytes each)
 enum {
-  B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages, B_V_FULL = B_K_EMPTY + kStages,
-  B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages, B_P_FULL = B_S_FULL + 2,
-  B_P_FREE = B_P_FULL + 2, B_DONE = B_P_FREE + 2, B_COUNT
+  B_Q16 = 0, B_Q8, B_Q4, B_SFQ, B_QFREE, B_S_FREE, B_K_FULL, B_K_EMPTY = B_K_FULL + kStages,
+  B_V_FULL = B_K_EMPTY + kStages, B_V_EMPTY = B_V_FULL + kStages, B_S_FULL = B_V_EMPTY + kStages,
+  B_P_FULL = B_S_FULL + 2, B_P_FREE = B_P_FULL + 2, B_DONE = B_P_FREE + 2, B_COUNT
 };
-static_assert(B_COUNT * 8 <= 512, "barrier area");
+static_assert(B_COUNT * 8 <= 256, "barrier area");
 
 struct TcArgs {
   const uint32_t* plist;  // [BH][npairs][2*nb]
@@ -185,6 +187,19 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 // 2^k for an integer-valued float k <= 127 (exact; 0 below the normal range)
 __device__ __forceinline__ float pow2i(float k) { return k > -127.0f ? __int_as_float(((int)k + 127) << 23) : 0.0f; }
+// Twice the sum of the eight e2m1 values packed in w (non-negative codes):
+// a byte permute looks up 2|v| for four codes at a time (0 1 2 3 4 6 8 12),
+// a byte dot product with ones adds them.
+__device__ __forceinline__ int e2m1_sum2(uint32_t w, int acc) {
+  constexpr uint32_t kLo = 0x03020100u, kHi = 0x0C080604u;
+  acc = __dp4a(__byte_perm(kLo, kHi, w & 0xffffu), 0x01010101u, (unsigned)acc);
+  return (int)__dp4a(__byte_perm(kLo, kHi, w >> 16), 0x01010101u, (unsigned)acc);
+}
+// value of a ue4m3 scale: 2^(e-7) (1 + m/8), or m 2^-9 when e = 0
+__device__ __forceinline__ float ue4m3_value(uint32_t sf) {
+  const uint32_t ex = sf >> 3, mt = sf & 7u;
+  return ex ? __uint_as_float(((ex + 120u) << 23) | (mt << 20)) : (float)mt * (1.0f / 512.0f);
+}
 
 // Items: kb | inA << 16 | inB << 17 | kind << 18 | full << 20 (the key block
 // has no padding slot).
@@ -213,18 +228,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                TcArgs A) {
   using SM = Smem<D>;
   constexpr int H = SM::H;
-  constexpr int DH = D / 2;  // channels per thread
   // a CTA that timed out raised the status word: later CTAs skip their work
   if (*reinterpret_cast<volatile const int*>(A.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s0 = (uint32_t)__cvta_generic_to_shared(smem);
-  const int bh = (int)(blockIdx.x / (unsigned)A.npairs), pair = (int)(blockIdx.x - (unsigned)bh * A.npairs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this warp's tile: its query-block pair, shared-memory half and TMEM columns
+  const int t = warp < kIssueWarp0 ? warp / kSoftmaxWarps : (warp - kIssueWarp0) >> 1;
+  const long long gi = (long long)kTiles * blockIdx.x + t;
+  const bool active = gi < (long long)A.npairs * g.BH;
+  const int bh = active ? (int)(gi / A.npairs) : 0, pair = active ? (int)(gi - (long long)bh * A.npairs) : 0;
+  uint8_t* ts = smem + t * SM::TILE;
+  const uint32_t s0t = s0 + t * SM::TILE;
   const int qa = 2 * pair, qb = (2 * pair + 1 < g.nb) ? 2 * pair + 1 : -1;
   const size_t prow = (size_t)bh * A.npairs + pair;
-  const int4 pc = kDense ? make_int4(g.nb, 0, 0, 0) : *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
-  const int n16 = pc.x, n8 = pc.y, n4 = pc.z;
+  const int4 pc = !active ? make_int4(0, 0, 0, 0)
+                 : kDense ? make_int4(g.nb, 0, 0, 0) : *reinterpret_cast<const int4*>(A.pcnt + prow * 4);
+  // one key block per unit: units [0, nu16) 16-bit, [nu16, nu8) INT8, [nu8, nu) 4-bit
+  const int nu16 = pc.x, nu8 = pc.x + pc.y, nu = pc.x + pc.y + pc.z;
   const uint32_t* items = kDense ? nullptr : A.plist + prow * (size_t)(2 * g.nb);
   const uint32_t spin = A.spin;
   // entry i of the pair's list; in dense mode key block i, kept by both query
@@ -234,161 +256,146 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     return (uint32_t)i | (1u << 16) | ((2 * pair + 1 < g.nb ? 1u : 0u) << 17) |
            ((uint32_t)((i + 1) * 64 <= g.N) << 20);
   };
-  auto bar = [&](int i) { return s0 + SM::BAR + 8u * (uint32_t)i; };
+  auto bar = [&](int i) { return s0t + SM::BAR + 8u * (uint32_t)i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + SM::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC + 8);
   // 1 / (1 + m/8) for m = 0..7, then 1 / m (0 for m = 0): reciprocals of e4m3 scales
   float* rcp_tab = reinterpret_cast<float*>(smem + SM::MISC + 64);
-  float* vsc = reinterpret_cast<float*>(smem + SM::VS);  // [4][D] channel factors (VS_*)
+  float* vsc = reinterpret_cast<float*>(ts + SM::VS);  // [4][D] channel factors (VS_*)
   if (threadIdx.x < 16)
     rcp_tab[threadIdx.x] = threadIdx.x < 8 ? 8.0f / (float)(8 + threadIdx.x)
                                            : (threadIdx.x > 8 ? 1.0f / (float)(threadIdx.x - 8) : 0.f);
 
-  // units: each phase takes its items (key blocks) two at a time, in list order
-  const int nu16 = (n16 + 1) / 2;
-  const int nu8 = nu16 + (n8 + 1) / 2;  // INT8 units end here, 4-bit units follow
-  const int nu = nu8 + (n4 + 1) / 2;
-  auto unit_items = [&](int u, int& i0, int& cnt) {
-    if (u < nu16) { i0 = 2 * u; cnt = min(2, n16 - i0); }
-    else if (u < nu8) { i0 = n16 + 2 * (u - nu16); cnt = min(2, n16 + n8 - i0); }
-    else { i0 = n16 + n8 + 2 * (u - nu8); cnt = min(2, n16 + n8 + n4 - i0); }
-  };
-
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_Q16), 1);
-    mbar_init(bar(B_Q8), 1);
-    mbar_init(bar(B_Q4), 1);
-    mbar_init(bar(B_SFQ), 4);  // warps 0-3 wrote Q's and the ones tile's scale factors
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(B_K_FULL + s), 1); mbar_init(bar(B_K_EMPTY + s), 1);
-      mbar_init(bar(B_V_FULL + s), 1); mbar_init(bar(B_V_EMPTY + s), 1);
+    for (int tt = 0; tt < kTiles; ++tt) {
+      auto tbar = [&](int i) { return s0 + tt * SM::TILE + SM::BAR + 8u * (uint32_t)i; };
+      mbar_init(tbar(B_Q16), 1);
+      mbar_init(tbar(B_Q8), 1);
+      mbar_init(tbar(B_Q4), 1);
+      mbar_init(tbar(B_SFQ), kSoftmaxWarps);     // each softmax warp wrote Q's scale factors in its lanes
+      mbar_init(tbar(B_QFREE), 1);               // the last 16-bit score MMA (the last reader of Q16) completed
+      mbar_init(tbar(B_S_FREE), kSoftmaxWarps);  // per 4-bit unit: its scores were read
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(tbar(B_K_FULL + s), 1); mbar_init(tbar(B_K_EMPTY + s), 1);
+        mbar_init(tbar(B_V_FULL + s), 1); mbar_init(tbar(B_V_EMPTY + s), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(tbar(B_S_FULL + b), 1);
+        mbar_init(tbar(B_P_FULL + b), kSoftmaxWarps);  // per unit parity: P of unit u written
+        mbar_init(tbar(B_P_FREE + b), 1);              // the P·V of unit u has completed
+      }
+      mbar_init(tbar(B_DONE), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(B_S_FULL + b), 1);
-      mbar_init(bar(B_P_FULL + b), kSoftmaxWarps);  // per unit parity: P of unit u written
-      mbar_init(bar(B_P_FREE + b), 1);              // the P·V of unit u has completed
-    }
-    mbar_init(bar(B_DONE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) tmem_alloc(s0 + SM::MISC, 512);
-  if (!kDense) {
-    for (int c = threadIdx.x; c < D; c += kThreads) {
-      const float sv = n8 > 0 ? A.v_s8[(size_t)bh * D + c] : 0.f, gv = n4 > 0 ? A.v_g4[(size_t)bh * D + c] : 0.f;
+  if (warp == kIssueWarp0 + 1) tmem_alloc(s0 + SM::MISC, kTmemCols);
+  if (!kDense && warp < kIssueWarp0) {
+    // each softmax warpgroup fills its own tile's channel factors
+    for (int c = threadIdx.x & 127; c < D; c += 128) {
+      const float sv = nu8 > nu16 ? A.v_s8[(size_t)bh * D + c] : 0.f, gv = nu > nu8 ? A.v_g4[(size_t)bh * D + c] : 0.f;
       vsc[VS_TO8 * D + c] = sv > 0.f ? 255.0f / sv : 1.0f;
       vsc[VS_FROM8 * D + c] = sv > 0.f ? sv / 255.0f : 1.0f;
       vsc[VS_TO4 * D + c] = gv > 0.f ? kP4Range / gv : 1.0f;
       vsc[VS_FROM4 * D + c] = gv > 0.f ? gv / kP4Range : 1.0f;
     }
-    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + SM::ONES);
-    for (int i = threadIdx.x; i < 512; i += kThreads) ones[i] = kOnesE2m1;
-    fence_async_smem();  // the ones tile is read by the tensor core
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = misc[0];
+  const uint32_t tcol = tbase + (uint32_t)t * kTileCols;  // this tile's TMEM columns
 
   const int t_of = g.nry * g.nrx;  // blocks per frame
   auto box = [&](int blk, int& cx, int& cy, int& cf) {
-    const int t = blk / t_of, rem = blk - t * t_of;
+    const int tf = blk / t_of, rem = blk - tf * t_of;
     const int ry = rem / g.nrx, rx = rem - ry * g.nrx;
-    cx = rx * g.rw; cy = ry * g.rh; cf = bh * g.T + t;
+    cx = rx * g.rw; cy = ry * g.rh; cf = bh * g.T + tf;
   };
 
-  if (warp >= kSoftmaxWarps) {
-  // the third warpgroup: producer, MMA issuer and two idle warps
-  setmaxnreg_dec<kRegsIssue>();
-  if (warp == kProducerWarp) {
+  if (warp >= kIssueWarp0) {
+  // the third warpgroup: each tile's TMA producer and MMA issuer
+  if (((warp - kIssueWarp0) & 1) == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (elect_one()) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
       int cx, cy, cf;
-      const bool q16 = n16 > 0, q8 = n8 > 0, q4 = n4 > 0;
+      const bool q16 = nu16 > 0, q8 = nu8 > nu16, q4 = nu > nu8;
       if (q16) {
         mbar_expect_tx(bar(B_Q16), (qb >= 0 ? 2u : 1u) * 128u * D);
         box(qa, cx, cy, cf);
-        for (int h = 0; h < H; ++h) tma_load_4d(s0 + SM::Q16 + h * 16384, &tmQ, bar(B_Q16), 64 * h, cx, cy, cf);
+        for (int h = 0; h < H; ++h) tma_load_4d(s0t + SM::Q + h * 16384, &tmQ, bar(B_Q16), 64 * h, cx, cy, cf);
         if (qb >= 0) {
           box(qb, cx, cy, cf);
           for (int h = 0; h < H; ++h)
-            tma_load_4d(s0 + SM::Q16 + h * 16384 + 8192, &tmQ, bar(B_Q16), 64 * h, cx, cy, cf);
+            tma_load_4d(s0t + SM::Q + h * 16384 + 8192, &tmQ, bar(B_Q16), 64 * h, cx, cy, cf);
         }
       }
-      if (q8) {
-        mbar_expect_tx(bar(B_Q8), (qb >= 0 ? 2u : 1u) * 64u * D);
-        tma_load_2d(s0 + SM::Q8, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qa) * 64);
-        if (qb >= 0) tma_load_2d(s0 + SM::Q8 + 64 * D, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qb) * 64);
-      }
-      if (q4) {
-        mbar_expect_tx(bar(B_Q4), (qb >= 0 ? 2u : 1u) * 32u * D);
-        tma_load_2d(s0 + SM::Q4, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qa) * 64);
-        if (qb >= 0) tma_load_2d(s0 + SM::Q4 + 32 * D, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qb) * 64);
-      }
+      // Q8 and Q4 go into Q16's buffer once its last reader has completed
+      bool qlow = !(q8 || q4);
       // K of a unit is needed first (scores) and released first; V waits for
       // the P·V two units back.  Issue whichever ring has room, K first.
       int kn = 0, vn = 0;
       int last_k[kStages] = {-1, -1}, last_v[kStages] = {-1, -1};  // last unit loaded into each slot
       uint32_t idle = 0;
-      while (kn < nu || vn < nu) {
+      while (kn < nu || vn < nu || !qlow) {
         bool progressed = false;
+        if (!qlow && (!q16 || mbar_test(bar(B_QFREE), 0))) {
+          if (q8) {
+            mbar_expect_tx(bar(B_Q8), (qb >= 0 ? 2u : 1u) * 64u * D);
+            tma_load_2d(s0t + SM::Q, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qa) * 64);
+            if (qb >= 0) tma_load_2d(s0t + SM::Q + 64 * D, &tmQ8, bar(B_Q8), 0, (bh * g.nb + qb) * 64);
+          }
+          if (q4) {
+            mbar_expect_tx(bar(B_Q4), (qb >= 0 ? 2u : 1u) * 32u * D);
+            tma_load_2d(s0t + SM::Q + SM::Q4OFF, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qa) * 64);
+            if (qb >= 0) tma_load_2d(s0t + SM::Q + SM::Q4OFF + 32 * D, &tmQ4, bar(B_Q4), 0, (bh * g.nb + qb) * 64);
+          }
+          qlow = true;
+          progressed = true;
+        }
         if (kn < nu && (kn < kStages || mbar_test(bar(B_K_EMPTY + kn % kStages), ((kn / kStages) - 1) & 1))) {
-          int i0, cnt;
-          unit_items(kn, i0, cnt);
-          const uint32_t dst = s0 + SM::KR + (kn % kStages) * SM::STAGE;
+          const int kb = item_kb(item_at(kn));
+          const uint32_t dst = s0t + SM::KR + (kn % kStages) * SM::STAGE;
           const uint32_t fb = bar(B_K_FULL + kn % kStages);
           if (kn == 0 && (int)blockIdx.x == A.poison) {
             // test hook: this load is never issued, so its consumers' bounded waits expire
           } else if (kn < nu16) {
-            mbar_expect_tx(fb, 128u * D * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t) {
-              box(item_kb(item_at(i0 + t)), cx, cy, cf);
-              for (int h = 0; h < H; ++h) tma_load_4d(dst + h * 16384 + t * 8192, &tmK, fb, 64 * h, cx, cy, cf);
-            }
+            mbar_expect_tx(fb, 128u * D);
+            box(kb, cx, cy, cf);
+            for (int h = 0; h < H; ++h) tma_load_4d(dst + h * 8192, &tmK, fb, 64 * h, cx, cy, cf);
             last_k[kn % kStages] = kn;
           } else if (kn < nu8) {
-            mbar_expect_tx(fb, 64u * D * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t)
-              tma_load_2d(dst + t * 64 * D, &tmK8, fb, 0, (bh * g.nb + item_kb(item_at(i0 + t))) * 64);
+            mbar_expect_tx(fb, 64u * D);
+            tma_load_2d(dst, &tmK8, fb, 0, (bh * g.nb + kb) * 64);
             last_k[kn % kStages] = kn;
           } else {
-            mbar_expect_tx(fb, (32u * D + H * kSfAtomBytes) * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t) {
-              const size_t kl = (size_t)bh * g.nb + item_kb(item_at(i0 + t));
-              tma_load_2d(dst + t * 32 * D, &tmK4, fb, 0, (int)(kl * 64));
-              bulk_load(dst + SM::SL_SF + t * H * kSfAtomBytes, A.k_sf4 + kl * H * kSfAtomBytes, H * kSfAtomBytes,
-                        fb);
-            }
+            const size_t kl = (size_t)bh * g.nb + kb;
+            mbar_expect_tx(fb, 32u * D + H * kSfAtomBytes);
+            tma_load_2d(dst, &tmK4, fb, 0, (int)(kl * 64));
+            bulk_load(dst + SM::SL_SF, A.k_sf4 + kl * H * kSfAtomBytes, H * kSfAtomBytes, fb);
             last_k[kn % kStages] = kn;
           }
           ++kn;
           progressed = true;
         }
         if (vn < kn && (vn < kStages || mbar_test(bar(B_V_EMPTY + vn % kStages), ((vn / kStages) - 1) & 1))) {
-          int i0, cnt;
-          unit_items(vn, i0, cnt);
-          const uint32_t dst = s0 + SM::VR + (vn % kStages) * SM::STAGE;
+          const int kb = item_kb(item_at(vn));
+          const uint32_t dst = s0t + SM::VR + (vn % kStages) * SM::STAGE;
           const uint32_t fb = bar(B_V_FULL + vn % kStages);
           if (vn < nu16) {
-            mbar_expect_tx(fb, 128u * D * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t) {
-              box(item_kb(item_at(i0 + t)), cx, cy, cf);
-              for (int h = 0; h < H; ++h) tma_load_4d(dst + (t * H + h) * 8192, &tmV, fb, 64 * h, cx, cy, cf);
-            }
+            mbar_expect_tx(fb, 128u * D);
+            box(kb, cx, cy, cf);
+            for (int h = 0; h < H; ++h) tma_load_4d(dst + h * 8192, &tmV, fb, 64 * h, cx, cy, cf);
           } else if (vn < nu8) {
             // the INT8 codes as bf16 values, [64 slots][D] per block: the 16-bit tile layout
-            mbar_expect_tx(fb, 128u * D * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t)
-              for (int h = 0; h < H; ++h)
-                tma_load_2d(dst + (t * H + h) * 8192, &tmV8, fb, 64 * h, (bh * g.nb + item_kb(item_at(i0 + t))) * 64);
+            mbar_expect_tx(fb, 128u * D);
+            for (int h = 0; h < H; ++h) tma_load_2d(dst + h * 8192, &tmV8, fb, 64 * h, (bh * g.nb + kb) * 64);
           } else {
-            mbar_expect_tx(fb, (32u * D + kSfAtomBytes) * (uint32_t)cnt);
-            for (int t = 0; t < cnt; ++t) {
-              const size_t kl = (size_t)bh * g.nb + item_kb(item_at(i0 + t));
-              tma_load_2d(dst + t * 32 * D, &tmV4, fb, 0, (int)(kl * D));
-              bulk_load(dst + SM::SL_SF + t * kSfAtomBytes, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
-            }
+            const size_t kl = (size_t)bh * g.nb + kb;
+            mbar_expect_tx(fb, 32u * D + kSfAtomBytes);
+            tma_load_2d(dst, &tmV4, fb, 0, (int)(kl * D));
+            bulk_load(dst + SM::SL_SF, A.v_sf4 + kl * kSfAtomBytes, kSfAtomBytes, fb);
           }
           last_v[vn % kStages] = vn;
           ++vn;
@@ -405,30 +412,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // every copy this CTA issued lands before the CTA may leave (bounded)
       if (q16) (void)mbar_wait(bar(B_Q16), 0, spin);
-      if (q8) (void)mbar_wait(bar(B_Q8), 0, spin);
-      if (q4) (void)mbar_wait(bar(B_Q4), 0, spin);
+      if (qlow && q8) (void)mbar_wait(bar(B_Q8), 0, spin);
+      if (qlow && q4) (void)mbar_wait(bar(B_Q4), 0, spin);
       for (int s = 0; s < kStages; ++s) {
         if (last_k[s] >= 0) (void)mbar_wait(bar(B_K_FULL + s), (uint32_t)(last_k[s] / kStages) & 1u, spin);
         if (last_v[s] >= 0) (void)mbar_wait(bar(B_V_FULL + s), (uint32_t)(last_v[s] / kStages) & 1u, spin);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else {
     // ---------------------------------------------------------------- MMA scheduler
     if (elect_one()) {
-      const uint32_t id16n128 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 128);
-      const uint32_t id16n64 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 64);
+      const uint32_t id16 = idesc(kDF32, kFmtBF16, kFmtBF16, false, false, 128, 64);
       const uint32_t idpv = idesc(kDF32, kFmtBF16, kFmtBF16, false, true, 128, D);
-      const uint32_t id8n64 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
-      const uint32_t id8n128 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 128);
-      const uint32_t id4s = idesc_f4(128, 64), id4pv = idesc_f4(128, D), id4l = idesc_f4(128, 64);
+      const uint32_t id8 = idesc(kDS32, kFmtS8, kFmtS8, false, false, 128, 64);
+      const uint32_t id4s = idesc_f4(128, 64), id4pv = idesc_f4(128, D);
       constexpr uint32_t kSbo8 = 8u * D;                       // INT8 rows of D bytes
       constexpr Swizzle kSw8 = D == 128 ? SW_128 : SW_64;
       constexpr uint32_t kSbo4 = 4u * D;                       // NVFP4 rows of D/2 bytes
       constexpr Swizzle kSw4 = D == 128 ? SW_64 : SW_32;
-      bool f4_ready = false;  // Q4 loaded and its scales in TMEM
+      bool q16_ready = nu16 == 0, q8_ready = nu8 == nu16, f4_ready = nu == nu8;
       bool ok = true;
-      if (n16 > 0) ok = ok && mbar_wait(bar(B_Q16), 0, spin);
-      if (n8 > 0) ok = ok && mbar_wait(bar(B_Q8), 0, spin);
       int sn = 0, pn = 0;  // next unit for S, next unit for P·V
       uint32_t idle = 0;
       // the P·V of unit j (and every MMA before it) has completed
@@ -437,44 +440,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         bool progressed = false;
         if (sn < nu) {
           const int s = sn % kStages, b = sn & 1;
-          const bool f4 = sn >= nu8;
-          if (f4 && !f4_ready) f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
-          // a score buffer is free once the P·V of the unit two back completed
-          // (its P sat in the buffer, or its scores were read before its P)
-          if ((!f4 || f4_ready) && pv_done(sn - 2) && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1)) {
+          bool can;
+          if (sn < nu16) {
+            if (!q16_ready) q16_ready = mbar_test(bar(B_Q16), 0);
+            // a score buffer is free once the P·V of the unit two back (whose P sat in it) completed
+            can = q16_ready && pv_done(sn - 2);
+          } else if (sn < nu8) {
+            if (!q8_ready) q8_ready = mbar_test(bar(B_Q8), 0);
+            can = q8_ready && pv_done(sn - 2);
+          } else {
+            // Q4 landed and the softmax wrote Q's scale factors, after every
+            // earlier P·V completed; afterwards the single 4-bit score buffer
+            // is free once the softmax has read the previous unit's scores
+            if (!f4_ready) f4_ready = mbar_test(bar(B_Q4), 0) && mbar_test(bar(B_SFQ), 0);
+            can = f4_ready && (sn == nu8 || mbar_test(bar(B_S_FREE), (uint32_t)(sn - 1 - nu8) & 1u));
+          }
+          if (can && mbar_test(bar(B_K_FULL + s), (sn / kStages) & 1)) {
             tc_fence_after();
-            const uint32_t st = s0 + SM::KR + s * SM::STAGE;
-            const uint32_t sd = tbase + TM_S + b * 128u;
-            int i0, cnt;
-            unit_items(sn, i0, cnt);
+            const uint32_t st = s0t + SM::KR + s * SM::STAGE;
             if (sn < nu16) {
-              const uint32_t id = cnt == 2 ? id16n128 : id16n64;
+              const uint32_t sd = tcol + TM_S + 64u * b;
 #pragma unroll
               for (int k = 0; k < D / 16; ++k) {
                 const int h = k >> 2, kk = k & 3;
-                mma_f16(sd, smem_desc(s0 + SM::Q16 + h * 16384 + kk * 32, 16, 1024, SW_128),
-                        smem_desc(st + h * 16384 + kk * 32, 16, 1024, SW_128), id, k > 0 ? 1u : 0u);
+                mma_f16(sd, smem_desc(s0t + SM::Q + h * 16384 + kk * 32, 16, 1024, SW_128),
+                        smem_desc(st + h * 8192 + kk * 32, 16, 1024, SW_128), id16, k > 0 ? 1u : 0u);
               }
             } else if (sn < nu8) {
-              const uint32_t id = cnt == 2 ? id8n128 : id8n64;
+              const uint32_t sd = tcol + TM_S + 64u * b;
 #pragma unroll
               for (int kk = 0; kk < D / 32; ++kk)
-                mma_i8(sd, smem_desc(s0 + SM::Q8 + kk * 32, 16, kSbo8, kSw8), smem_desc(st + kk * 32, 16, kSbo8, kSw8),
-                       id, kk > 0 ? 1u : 0u);
+                mma_i8(sd, smem_desc(s0t + SM::Q + kk * 32, 16, kSbo8, kSw8), smem_desc(st + kk * 32, 16, kSbo8, kSw8),
+                       id8, kk > 0 ? 1u : 0u);
             } else {
-              for (int t = 0; t < cnt; ++t) {
+              const uint32_t sfk = tcol + TM_SFK + 8u * b;
 #pragma unroll
-                for (int c = 0; c < H; ++c) {
-                  const uint32_t sfk = tbase + TM_SFK + 8 * t + 4 * c;
-                  tc_cp_atom(sfk, st + SM::SL_SF + (t * H + c) * kSfAtomBytes);
-                  mma_f4(sd + 64 * t, smem_desc(s0 + SM::Q4 + 32 * c, 16, kSbo4, kSw4),
-                         smem_desc(st + t * 32 * D + 32 * c, 16, kSbo4, kSw4), id4s, c > 0 ? 1u : 0u,
-                         tbase + TM_SFQ + 4 * c, sfk);
-                }
+              for (int c = 0; c < H; ++c) {
+                tc_cp_atom(sfk + 4 * c, st + SM::SL_SF + c * kSfAtomBytes);
+                mma_f4(tcol + TM_S4, smem_desc(s0t + SM::Q + SM::Q4OFF + 32 * c, 16, kSbo4, kSw4),
+                       smem_desc(st + 32 * c, 16, kSbo4, kSw4), id4s, c > 0 ? 1u : 0u, tcol + TM_SFQ + 4 * c,
+                       sfk + 4 * c);
               }
             }
             mma_commit(bar(B_S_FULL + b));
             mma_commit(bar(B_K_EMPTY + s));
+            if (sn == nu16 - 1) mma_commit(bar(B_QFREE));
             ++sn;
             progressed = true;
           }
@@ -483,29 +493,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int s = pn % kStages;
           if (mbar_test(bar(B_V_FULL + s), (pn / kStages) & 1) && mbar_test(bar(B_P_FULL + (pn & 1)), (pn >> 1) & 1)) {
             tc_fence_after();
-            const uint32_t st = s0 + SM::VR + s * SM::STAGE;
-            const uint32_t pt = tbase + TM_S + (pn & 1) * 128u;  // the unit's P (16-bit, INT8) in TMEM
-            int i0, cnt;
-            unit_items(pn, i0, cnt);
+            const uint32_t st = s0t + SM::VR + s * SM::STAGE;
             if (pn < nu8) {
               // 16-bit and INT8 units: P (bf16) from TMEM, V tiles MN-major bf16
-              for (int t = 0; t < cnt; ++t) {
+              const uint32_t pt = tcol + TM_S + 64u * (pn & 1);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_f16_ta(tbase + TM_O, pt + 64 * t + 8 * kk,
-                             smem_desc(st + t * H * 8192 + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
-              }
+              for (int kk = 0; kk < 4; ++kk)
+                mma_f16_ta(tcol + TM_O, pt + 8 * kk, smem_desc(st + kk * 2048, 8192, 1024, SW_128), idpv, 1u);
             } else {
-              const uint32_t pb = s0 + SM::P4 + (pn & 1) * SM::P4STRIDE;
-              for (int t = 0; t < cnt; ++t) {
-                const uint32_t sfv = tbase + TM_SFV + 4 * t, sfp = tbase + TM_SFP + 4 * t;
-                tc_cp_atom(sfv, st + SM::SL_SF + t * kSfAtomBytes);
-                tc_cp_atom(sfp, pb + SM::P4SF + t * kSfAtomBytes);
-                mma_f4(tbase + TM_O, smem_desc(pb + t * 4096, 16, 256, SW_32),
-                       smem_desc(st + t * 32 * D, 16, 256, SW_32), id4pv, 1u, sfp, sfv);
-                mma_f4(tbase + TM_L4, smem_desc(pb + t * 4096, 16, 256, SW_32),
-                       smem_desc(s0 + SM::ONES, 16, 256, SW_32), id4l, 1u, sfp, tbase + TM_SF1);
-              }
+              const uint32_t pb = s0t + SM::P4 + (pn & 1) * SM::P4STRIDE;
+              const uint32_t sfv = tcol + TM_SFV + 4u * (pn & 1), sfp = tcol + TM_SFP + 4u * (pn & 1);
+              tc_cp_atom(sfv, st + SM::SL_SF);
+              tc_cp_atom(sfp, pb + SM::P4SF);
+              mma_f4(tcol + TM_O, smem_desc(pb, 16, 256, SW_32), smem_desc(st, 16, 256, SW_32), id4pv, 1u, sfp, sfv);
             }
             mma_commit(bar(B_P_FREE + (pn & 1)));
             mma_commit(bar(B_V_EMPTY + s));
@@ -526,88 +526,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   }
   } else {
-    setmaxnreg_inc<kRegsSoftmax>();
     // ---------------------------------------------------------------- softmax warps 0-7
-    const int q4 = warp & 3, sub = warp >> 2;
-    const int hh = lane >> 4;                       // key block of a unit / channel half
-    const int row = q4 * 32 + sub * 16 + (lane & 15);  // TMEM lane and tile row
-    const bool in_b = q4 >= 2;
+    const int row = threadIdx.x & 127;               // TMEM lane and tile row
+    const int wq = warp & 3;                         // lane quarter
+    const bool in_b = row >= 64;
     const int qrow_blk = in_b ? qb : qa;
-    const uint32_t tl = tbase + ((uint32_t)(q4 * 32 + sub * 16) << 16);  // this warp's 16 lanes
+    const uint32_t tl = tcol + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
     const float sl2 = kLog2e * rsqrtf((float)D);
-    const float sq = (!kDense && n8 > 0 && qrow_blk >= 0) ? A.q_s8[(size_t)bh * g.nb + qrow_blk] : 0.f;
+    const float sq = (!kDense && nu8 > nu16 && qrow_blk >= 0) ? A.q_s8[(size_t)bh * g.nb + qrow_blk] : 0.f;
     const unsigned FULL = 0xffffffffu;
     // the P·V of unit v (and every MMA before it) has completed
     auto pfree_wait = [&](int v) -> bool {
       return v < 0 || mbar_wait(bar(B_P_FREE + (v & 1)), (uint32_t)(v >> 1) & 1u, spin);
     };
     float ref = -INFINITY;    // O's reference per row: an integer, log2 units (the shared statistics)
-    float l = 0.f;            // this thread's part of the row sum, relative to 2^ref
+    float l = 0.f;            // the row sum, relative to 2^ref
     float x_run = -INFINITY;  // running row max (log2 units) over every unit so far
     bool ok = true;
 #pragma unroll
-    for (int c = 0; c < DH; c += 32) tmem_fill16x2_x32<DH>(tl + TM_O + c, 0u);  // O starts at zero
-    if (n4 > 0) {
-      tmem_fill16x2_x32<32>(tl + TM_L4, 0u);  // so do the 4-bit row sums
-      if (warp < 4) {
-        // warp w writes lane quarter w (32x32b shape): per 64-channel chunk the
-        // scale atoms of both query blocks (rows i, i+32 | i+64, i+96), and
-        // the ones tile's scales (all 1)
-        const uint32_t tq = tbase + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-        for (int c = 0; c < H; ++c) {
-          uint32_t w[4];
-          const uint8_t* sa = A.q_sf4 + ((size_t)bh * g.nb + qa) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
-          w[0] = *reinterpret_cast<const uint32_t*>(sa);
-          w[1] = *reinterpret_cast<const uint32_t*>(sa + 4);
-          if (qb >= 0) {
-            const uint8_t* sbp = A.q_sf4 + ((size_t)bh * g.nb + qb) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
-            w[2] = *reinterpret_cast<const uint32_t*>(sbp);
-            w[3] = *reinterpret_cast<const uint32_t*>(sbp + 4);
-          } else {
-            w[2] = w[3] = 0u;
-          }
-          tmem_st4(tq + TM_SFQ + 4 * c, w);
-        }
-        const uint32_t one[4] = {kOneE4m3x4, kOneE4m3x4, kOneE4m3x4, kOneE4m3x4};
-        tmem_st4(tq + TM_SF1, one);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_SFQ));
-      }
-    }
+    for (int c = 0; c < D; c += 32) tmem_fill32(tl + TM_O + c, 0u);  // O starts at zero
     tmem_wait_st();
     // item entries (and INT8 key scales) are loaded one unit ahead, so no unit
     // starts by waiting on global memory
-    auto item_for = [&](int v) -> uint32_t {
-      if (v >= nu) return 0u;
-      int i0v, cntv;
-      unit_items(v, i0v, cntv);
-      return hh < cntv ? item_at(i0v + hh) : 0u;
-    };
+    auto item_for = [&](int v) -> uint32_t { return v < nu ? item_at(v) : 0u; };
     auto sk_for = [&](int v, uint32_t ev) -> float {
       return (v >= nu16 && v < nu8) ? A.k_s8[(size_t)bh * g.nb + item_kb(ev)] : 0.f;
     };
     uint32_t e_next = item_for(0);
     float sk_next = sk_for(0, e_next);
-    auto member_of = [&](uint32_t e, int u) -> bool {
-      int i0v, cntv;
-      unit_items(u, i0v, cntv);
-      return hh < cntv && (((e >> (in_b ? 17 : 16)) & 1u) != 0);
-    };
-    // O (this thread's channels) times a per-row factor a and per-channel
-    // factors ch[] (ch == nullptr: none); the MMAs that write O have completed
+    auto member_of = [&](uint32_t e) -> bool { return ((e >> (in_b ? 17 : 16)) & 1u) != 0; };
+    // O (this thread's row) times a per-row factor a and per-channel factors
+    // ch[] (ch == nullptr: none); the MMAs that write O have completed
     auto scale_o = [&](float a, const float* ch) {
 #pragma unroll 1
-      for (int c = 0; c < DH; c += 32) {
+      for (int c = 0; c < D; c += 32) {
         uint32_t orr[32];
-        tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
+        tmem_ld32(tl + TM_O + c, orr);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i)
           orr[i] = __float_as_uint(__uint_as_float(orr[i]) * (ch ? a * ch[c + i] : a));
-        tmem_st16x2_x32<DH>(tl + TM_O + c, orr);
+        tmem_st32(tl + TM_O + c, orr);
       }
       tmem_wait_st();
     };
@@ -629,7 +588,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
         scale_o(a, nullptr);
       }
-      tmem_st16x2_x32<64>(sb, pw);
+      tmem_st32(sb, pw);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -647,15 +606,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ================================================================ 16-bit phase
     for (int u = 0; ok && u < nu16; ++u) {
       if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-      const uint32_t sb = tl + TM_S + (u & 1) * 128u;
+      const uint32_t sb = tl + TM_S + 64u * (u & 1);
       if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1, spin))) { ok = false; break; }
       tc_fence_after();
       const uint32_t e = e_next;
-      const bool member = member_of(e, u);
+      const bool member = member_of(e);
       e_next = item_for(u + 1);
       uint32_t sr[64];
-      tmem_ld16x2_x32<64>(sb, sr);
-      tmem_ld16x2_x32<64>(sb + 32, sr + 32);
+      tmem_ld32(sb, sr);
+      tmem_ld32(sb + 32, sr + 32);
       tmem_wait_ld();
       float mx = -INFINITY;
       if (member) {
@@ -673,7 +632,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
       }
       sk_next = sk_for(u + 1, e_next);
-      const float um = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16)) * sl2;  // unit row max, log2 units
+      const float um = mx * sl2;  // the unit's row max, log2 units
       x_run = fmaxf(x_run, um);
       bool need_o;
       const float a = lazy_raise(um, need_o);
@@ -706,19 +665,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && nu8 > nu16) {
       // O goes to INT8 units (divided by the V channel scale sv/255)
       ok = boundary(nu16 - 1);
-      if (ok) scale_o(1.0f, vsc + VS_TO8 * D + hh * DH);
+      if (ok) scale_o(1.0f, vsc + VS_TO8 * D);
       for (int u = nu16; ok && u < nu8; ++u) {
         if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-        const uint32_t sb = tl + TM_S + (u & 1) * 128u;
+        const uint32_t sb = tl + TM_S + 64u * (u & 1);
         if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1, spin))) { ok = false; break; }
         tc_fence_after();
         const uint32_t e = e_next;
         const float sk = sk_next;
-        const bool member = member_of(e, u);
+        const bool member = member_of(e);
         e_next = item_for(u + 1);
         uint32_t sr[64];
-        tmem_ld16x2_x32<64>(sb, sr);
-        tmem_ld16x2_x32<64>(sb + 32, sr + 32);
+        tmem_ld32(sb, sr);
+        tmem_ld32(sb + 32, sr + 32);
         tmem_wait_ld();
         const unsigned long long vm = item_full(e) ? ~0ull : key_mask(g, item_kb(e));
         const bool full = vm == ~0ull;
@@ -739,7 +698,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           xh = (float)max(max(m4[0], m4[1]), max(m4[2], m4[3])) * sc;  // a member row has a real key
         }
         sk_next = sk_for(u + 1, e_next);
-        const float um = fmaxf(xh, __shfl_xor_sync(FULL, xh, 16));
+        const float um = xh;
         x_run = fmaxf(x_run, um);
         bool need_o;
         const float a = lazy_raise(um, need_o);
@@ -785,7 +744,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       // back to value units
       if (ok) ok = boundary(nu8 - 1);
-      if (ok) scale_o(1.0f, vsc + VS_FROM8 * D + hh * DH);
+      if (ok) scale_o(1.0f, vsc + VS_FROM8 * D);
     }
 
     // ================================================================ 4-bit phase
@@ -798,31 +757,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float a0 = (ref == -INFINITY || r0 == ref) ? 1.0f : pow2i(ref - r0);
       ref = r0;
       l *= a0;
-      if (ok) scale_o(a0, vsc + VS_TO4 * D + hh * DH);
-      // L4 (the quantised row sums, relative to 2^ref) joins l; rows in `sel` only
-      auto fold_l4 = [&](bool sel, float a) {
-        uint32_t lv;
-        tmem_ld16x2_x1<32>(tl + TM_L4, lv);
-        tmem_wait_ld();
-        if (sel && hh == 0) l = fmaf(__uint_as_float(lv), 1.0f / kP4Range, l);
-        if (sel) l *= a;
-        tmem_fill16x2_x32<32>(tl + TM_L4, sel ? 0u : lv);
-      };
+      if (ok) {
+        scale_o(a0, vsc + VS_TO4 * D);
+        // Q's scale factors into TMEM (the columns of the first score buffer,
+        // free now that every earlier P·V has completed): this warp writes its
+        // lane quarter, lane i the scales of rows i, i+32 (query block a) and
+        // i+64, i+96 (query block b) per 64-channel chunk
+        const uint32_t tq = tl;
+#pragma unroll
+        for (int c = 0; c < H; ++c) {
+          uint32_t w[4];
+          const uint8_t* sa = A.q_sf4 + ((size_t)bh * g.nb + qa) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+          w[0] = *reinterpret_cast<const uint32_t*>(sa);
+          w[1] = *reinterpret_cast<const uint32_t*>(sa + 4);
+          if (qb >= 0) {
+            const uint8_t* sbp = A.q_sf4 + ((size_t)bh * g.nb + qb) * H * kSfAtomBytes + c * kSfAtomBytes + lane * 16;
+            w[2] = *reinterpret_cast<const uint32_t*>(sbp);
+            w[3] = *reinterpret_cast<const uint32_t*>(sbp + 4);
+          } else {
+            w[2] = w[3] = 0u;
+          }
+          tmem_st4(tq + TM_SFQ + 4 * c, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SFQ));
+      }
       for (int u = nu8; ok && u < nu; ++u) {
         if ((u & 7) == 0 && __any_sync(FULL, *abort_flag != 0)) { ok = false; break; }
-        const uint32_t sb = tl + TM_S + (u & 1) * 128u;
+        const uint32_t sb = tl + TM_S4;
         if (!__all_sync(FULL, mbar_wait(bar(B_S_FULL + (u & 1)), (u >> 1) & 1, spin))) { ok = false; break; }
         tc_fence_after();
         const uint32_t e = e_next;
-        const bool member = member_of(e, u);
-        int i0, cnt;
-        unit_items(u, i0, cnt);
-        const bool present = hh < cnt;
+        const bool member = member_of(e);
         e_next = item_for(u + 1);
         uint32_t sr[64];
-        tmem_ld16x2_x32<64>(sb, sr);
-        tmem_ld16x2_x32<64>(sb + 32, sr + 32);
+        tmem_ld32(sb, sr);
+        tmem_ld32(sb + 32, sr + 32);
         tmem_wait_ld();
+        // the scores are in registers: the MMA warp may overwrite the buffer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_FREE));
         const unsigned long long vm = item_full(e) ? ~0ull : key_mask(g, item_kb(e));
         float mx = -INFINITY;
         if (member) {
@@ -839,18 +816,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               m4[q] = fmax3(m4[q], __uint_as_float(sr[i + 2 * q]), __uint_as_float(sr[i + 2 * q + 1]));
           mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;
         }
-        const float um = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));  // the unit's row maximum
-        // the reference rises to ceil(max) whenever the max exceeds it: O and
-        // the row sums are rescaled first, once the P·V of the unit before completed
+        const float um = mx;  // the unit's row maximum
+        // the reference rises to ceil(max) whenever the max exceeds it: O is
+        // rescaled first, once the P·V of the unit before completed
         const bool raise = um != -INFINITY && (ref == -INFINITY || um > ref);
         const float a = (raise && ref != -INFINITY) ? pow2i(ref - ceilf(um)) : 1.0f;
         if (__any_sync(FULL, raise)) {
           if (!__all_sync(FULL, pfree_wait(u - 1))) { ok = false; break; }
           tc_fence_after();
-          fold_l4(raise, a);
           scale_o(a, nullptr);
         }
-        if (raise) ref = ceilf(um);
+        if (raise) { l *= a; ref = ceilf(um); }
         uint32_t pw[8];
         uint32_t sfw = 0u;  // the row's four e4m3 P scales
 #pragma unroll
@@ -865,6 +841,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             sr[2 * i + 1] = __float_as_uint(fast_exp2(x1));
           }
           // NVFP4 of 2688 p over 16 consecutive keys: e4m3 scale from the microblock max / 6
+          float lq = 0.f;  // sum of the quantised weights, in units of 2688 / 2
 #pragma unroll
           for (int mbk = 0; mbk < 4; ++mbk) {
             float pm = 0.f;
@@ -877,6 +854,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const uint32_t ex = sf >> 3, mt = sf & 7u;
             const float inv_m = rcp_tab[ex ? mt : 8u + mt];
             const float rr = kP4Range * inv_m * __uint_as_float((ex ? 134u - ex : 136u) << 23);
+            int s2 = 0;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
               uint32_t w = 0;
@@ -886,31 +864,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 w |= cvt_e2m1x2(__uint_as_float(sr[k + 1]) * rr, __uint_as_float(sr[k]) * rr) << (8 * t);
               }
               pw[2 * mbk + q] = w;
+              s2 = e2m1_sum2(w, s2);
             }
+            lq = fmaf(ue4m3_value(sf), (float)s2, lq);
           }
+          l = fmaf(lq, 0.5f / kP4Range, l);
         }
         // P4 goes to shared memory buffer u&1, free once the P·V of unit u-2 completed
         if (u - 2 >= nu8 && !__all_sync(FULL, pfree_wait(u - 2))) { ok = false; break; }
-        if (present) {
-          uint8_t* pb = smem + SM::P4 + (u & 1) * SM::P4STRIDE + hh * 4096;
+        uint8_t* pb = ts + SM::P4 + (u & 1) * SM::P4STRIDE;
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-            *reinterpret_cast<uint4*>(pb + row * 32 + ((c ^ ((row >> 2) & 1)) * 16)) =
-                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-          *reinterpret_cast<uint32_t*>(smem + SM::P4 + (u & 1) * SM::P4STRIDE + SM::P4SF + hh * kSfAtomBytes +
-                                       (row & 31) * 16 + (row >> 5) * 4) = sfw;
-        }
+        for (int c = 0; c < 2; ++c)
+          *reinterpret_cast<uint4*>(pb + row * 32 + ((c ^ ((row >> 2) & 1)) * 16)) =
+              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        *reinterpret_cast<uint32_t*>(pb + SM::P4SF + (row & 31) * 16 + (row >> 5) * 4) = sfw;
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL + (u & 1)));
       }
-      // the phase's row sums join l and O returns to value units
+      // O returns to value units
       if (ok) ok = boundary(nu - 1);
-      if (ok) {
-        fold_l4(true, 1.0f);
-        scale_o(1.0f, vsc + VS_FROM4 * D + hh * DH);
-      }
+      if (ok) scale_o(1.0f, vsc + VS_FROM4 * D);
     }
     if (!ok) { raise_timeout(A.status); *abort_flag = 1; }
     // ---- epilogue: O / l in bf16, staged for the TMA store
@@ -919,16 +894,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // only the 16-bit phase ran: its last P·V completes before O is read
         if (!boundary(nu - 1)) { raise_timeout(A.status); *abort_flag = 1; }
       }
-      const float lt = l + __shfl_xor_sync(FULL, l, 16);
-      const float il = lt > 0.f ? 1.0f / lt : 0.f;
+      const float il = l > 0.f ? 1.0f / l : 0.f;
       const int r = row & 63;
-      uint8_t* ot = smem + SM::Q16 + (D == 128 ? hh * 16384 : 0) + (in_b ? 8192 : 0) + r * 128;
-      const int chunk0 = D == 128 ? 0 : 4 * hh;  // 16-byte chunk of this thread's first channel
 #pragma unroll
-      for (int c = 0; c < DH; c += 32) {
+      for (int c = 0; c < D; c += 32) {
         uint32_t orr[32];
-        tmem_ld16x2_x32<DH>(tl + TM_O + c, orr);
+        tmem_ld32(tl + TM_O + c, orr);
         tmem_wait_ld();
+        uint8_t* ot = ts + SM::Q + (c >> 6) * 16384 + (in_b ? 8192 : 0) + r * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t w[4];
@@ -938,7 +911,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                                       __uint_as_float(orr[8 * q + 2 * i + 1]) * il);
             w[i] = *reinterpret_cast<uint32_t*>(&hb);
           }
-          const int chunk = chunk0 + (c >> 3) + q;
+          const int chunk = ((c & 63) >> 3) + q;  // 16-byte chunk inside the 128-byte row
           *reinterpret_cast<uint4*>(ot + ((chunk ^ (r & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
@@ -947,7 +920,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && !*abort_flag) {
+  if ((threadIdx.x & 127) == 0 && warp < kIssueWarp0 && active && !*abort_flag) {
+    // the first thread of each softmax warpgroup stores its tile
     int cx, cy, cf;
     for (int blk = 0; blk < 2; ++blk) {
       const int qq = blk ? qb : qa;
@@ -955,7 +929,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       box(qq, cx, cy, cf);
       for (int h = 0; h < H; ++h)
         asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-                     ::"l"(&tmO), "r"(s0 + SM::Q16 + h * 16384 + blk * 8192), "r"(64 * h), "r"(cx), "r"(cy), "r"(cf)
+                     ::"l"(&tmO), "r"(s0t + SM::Q + h * 16384 + blk * 8192), "r"(64 * h), "r"(cx), "r"(cy), "r"(cf)
                      : "memory");
     }
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -963,11 +937,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) {
-    // every issued MMA has completed before the columns are released
-    (void)__all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, spin));
+  if (warp == kIssueWarp0 + 1) {
+    // every issued MMA of both tiles has completed before the columns are released
+    bool done = true;
+    for (int tt = 0; tt < kTiles; ++tt)
+      done = mbar_wait(s0 + tt * SM::TILE + SM::BAR + 8u * B_DONE, 0, spin) && done;
+    (void)__all_sync(0xffffffffu, done);
     tmem_relinquish();
-    tmem_dealloc(tbase, 512);
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 
@@ -1076,22 +1053,35 @@ bool map_bf16_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t col
 // path's; the dense entry point has no workspace to report through).
 __device__ int g_dense_status;
 
+// Kernel attributes: the dynamic shared memory (two tiles of about 110 KB)
+// and the largest shared-memory carveout.
+template <int D, bool kDense>
+cudaError_t configure_tc() {
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Smem<D>::BYTES);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_tc_kernel<D, kDense>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
+
 template <int D, bool kDense>
 cudaError_t launch_tc(const Geom& g, const CUtensorMap* maps, const TcArgs& A, cudaStream_t st) {
-  const long long ctas = (long long)A.npairs * g.BH;
+  // kTiles query-block pairs per CTA
+  const long long ctas = ((long long)A.npairs * g.BH + kTiles - 1) / kTiles;
   if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;
-  const int smem = (int)Smem<D>::BYTES;
-  // the register split needs the launch to hold kRegsLaunch per thread: a
-  // smaller allocation would leave the softmax warpgroups' increase waiting
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, kDense>);
+  cudaError_t e = configure_tc<D, kDense>();
   if (e != cudaSuccess) return e;
-  if ((uint32_t)fa.numRegs != kRegsLaunch) return cudaErrorNotSupported;
-  e = cudaFuncSetAttribute(attn_tc_kernel<D, kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  attn_tc_kernel<D, kDense><<<(unsigned)ctas, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                    maps[5], maps[6], maps[7], maps[8], maps[9], g, A);
+  attn_tc_kernel<D, kDense><<<(unsigned)ctas, kThreads, Smem<D>::BYTES, st>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], maps[8], maps[9], g, A);
   return cudaGetLastError();
+}
+
+template <int D, bool kDense>
+cudaError_t occupancy_tc(int* ctas_per_sm) {
+  cudaError_t e = configure_tc<D, kDense>();
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, attn_tc_kernel<D, kDense>, kThreads,
+                                                       Smem<D>::BYTES);
 }
 
 }  // namespace
@@ -1194,6 +1184,12 @@ cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* 
   A.spin = kDefaultSpin;
   A.poison = -1;
   return d == 128 ? launch_tc<128, true>(g, m, A, st) : launch_tc<64, true>(g, m, A, st);
+}
+
+cudaError_t attention_occupancy(int d, bool dense, int* ctas_per_sm) {
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
+  if (dense) return d == 128 ? occupancy_tc<128, true>(ctas_per_sm) : occupancy_tc<64, true>(ctas_per_sm);
+  return d == 128 ? occupancy_tc<128, false>(ctas_per_sm) : occupancy_tc<64, false>(ctas_per_sm);
 }
 
 cudaError_t dense_status(int* word, cudaStream_t st) {

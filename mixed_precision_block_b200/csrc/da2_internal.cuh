@@ -185,6 +185,8 @@ cudaError_t launch_attention(const Geom& g, const Layout& L, const void* q, cons
 cudaError_t launch_dense(int B, int H, int N, int d, const void* q, const void* k,
                          const void* v, void* out, cudaStream_t st);
 // Status word of the dense path: synchronises `st` and copies it to *word.
+// CTAs of the attention kernel (head dimension d, sparse or dense) an SM holds at once.
+cudaError_t attention_occupancy(int d, bool dense, int* ctas_per_sm);
 cudaError_t dense_status(int* word, cudaStream_t st);
 cudaError_t launch_pair_lists(const Geom& g, const Layout& L, void* ws, cudaStream_t st);
 // TMA: whether the driver's tensor-map encoder was found, and the 4-D view

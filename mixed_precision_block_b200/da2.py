@@ -26,7 +26,8 @@ VIEWS = ["PERM", "Q_AVG", "K_AVG", "Q_MAX", "K_MAX", "Q_I8", "K_I8", "Q_S8", "K_
          "Q_F4", "K_F4", "Q_SF4", "K_SF4", "V_I8", "V_S8", "V_F4", "V_SF4", "V_G4",
          "SCORES", "MAP", "LISTS", "COUNTS", "STATUS"]
 EXPORTS = ["da2_plan", "da2_prepare", "da2_draft_rank", "da2_rank_from_scores", "da2_attention",
-           "da2_dense_attention", "da2_dense_check_status", "da2_attention_wait_test", "da2_debug_view",
+           "da2_dense_attention", "da2_dense_check_status", "da2_attention_wait_test",
+           "da2_attention_occupancy", "da2_debug_view",
            "da2_rank_noalloc", "da2_check_status", "da2_host_bytes", "da2_forward_host", "da2_status_string"]
 NOALLOC_MAX_HEADS = 64  # DA2_NOALLOC_MAX_HEADS
 
@@ -66,6 +67,7 @@ _lib.da2_attention.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.da2_dense_attention.argtypes = [ctypes.c_int] * 4 + [_vp] * 5
 _lib.da2_dense_check_status.argtypes = [_vp]
 _lib.da2_attention_wait_test.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp, ctypes.c_int, ctypes.c_uint, _vp]
+_lib.da2_attention_occupancy.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
 _lib.da2_debug_view.argtypes = [_P, _vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_sz)]
 _lib.da2_rank_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
 _lib.da2_check_status.argtypes = [_P, _vp, _sz, _vp]
@@ -196,6 +198,13 @@ def da2_attention_wait_test(p, q, k, v, ws, out, withheld_cta, wait_polls, strea
     with da2_check_status)."""
     return _lib.da2_attention_wait_test(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel(),
                                         _ptr(out), int(withheld_cta), int(wait_polls), _stream(stream, ws))
+
+
+def da2_attention_occupancy(d, dense=False):
+    """CTAs of the attention kernel (head dimension d) that one SM holds at once."""
+    n = ctypes.c_int()
+    _check("da2_attention_occupancy", _lib.da2_attention_occupancy(int(d), 1 if dense else 0, ctypes.byref(n)))
+    return n.value
 
 
 def da2_debug_view(p, ws, which):

@@ -52,6 +52,15 @@ def _full_check(wl, heads=None, dense_ref=True):
     return outs
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dense", [False, True])
+def test_attention_cta_fits_an_sm(d, dense):
+    # one CTA per SM, holding two query-block pairs whose softmax warpgroups
+    # hide each other's latency: its registers, shared memory and launch
+    # attributes must admit it
+    assert da2.da2_attention_occupancy(d, dense) == 1
+
+
 def test_tiny_workload_all_stages():
     _full_check(WORKLOADS["tiny"])
 

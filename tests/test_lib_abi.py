@@ -93,6 +93,9 @@ def test_entry_points_check_workspace_and_pointers_before_launch(da2):
                                        None) == da2.DA2_ERR_ARG  # a zero wait bound
     assert lib.da2_check_status(ctypes.byref(p), None, big, None) == da2.DA2_ERR_WORKSPACE
     assert lib.da2_check_status(ctypes.byref(p), fake, big - 1, None) == da2.DA2_ERR_WORKSPACE
+    n = ctypes.c_int()
+    assert lib.da2_attention_occupancy(96, 0, ctypes.byref(n)) == da2.DA2_ERR_ARG
+    assert lib.da2_attention_occupancy(128, 0, None) == da2.DA2_ERR_ARG
 
 
 def test_workspace_views_are_disjoint_and_inside(da2):
