@@ -131,7 +131,7 @@ def whole_job_value(world, flops_per_rank, ms):
 
 def launches_per_call(info, d):
     """Kernels this library launches per call (its own kernels only)."""
-    v = 2 if (info.n8 or info.n4) else 0  # v_amax + pack_v
+    v = 1 if (info.n8 or info.n4) else 0  # the V preparation (absmax and codes in one kernel)
     prep = 1 + v
     draft = 2  # logits + mix (mix carries the first ranking histogram)
     rank = 1 + 8 + 7 + 1  # init, 8 selects, 7 histogram passes, assign

@@ -91,7 +91,10 @@ int da2_plan(const da2_problem* p, da2_plan_info* out);
  * block) and NVFP4 (e4m3 scale per 16 channels of a token).  V is quantised
  * per channel (INT8; NVFP4 with a per-channel fp32 scale and e4m3 scales per
  * 16 tokens) and transposed to [block][channel][token].  Formats the budget
- * does not use are not written.  q, k, v: device bf16 [B,H,N,d]. */
+ * does not use are not written.  q, k, v: device bf16 [B,H,N,d].  V crosses
+ * HBM about once: one persistent kernel merges a head's channel absmax and
+ * writes its codes one head later, from L2, after a bounded wait whose expiry
+ * sets the second status word (da2_check_status). */
 int da2_prepare(const da2_problem* p, const void* q, const void* k, const void* v,
                 void* ws, size_t ws_bytes, void* stream);
 
@@ -189,9 +192,11 @@ int da2_attention_occupancy(int d, int dense, int* ctas_per_sm);
  *   LISTS  uint16 [B*H][nb][nb] per query block: its 16-bit key blocks, then
  *          its 8-bit, then its 4-bit ones, each ascending
  *   COUNTS int32 [B*H][nb][4]   lengths of the three lists, 0
- *   STATUS int32 [1]            0, or 1 after a tensor-core attention call whose
- *                               bounded pipeline waits expired (its output is
- *                               then invalid); reset by every da2_attention */
+ *   STATUS int32 [2]            word 0: 0, or 1 after a tensor-core attention
+ *                               call whose bounded pipeline waits expired (its
+ *                               output is then invalid), reset by every
+ *                               da2_attention; word 1: the same for the V
+ *                               preparation, reset by every da2_prepare */
 enum {
   DA2_VIEW_PERM = 0,
   DA2_VIEW_Q_AVG, DA2_VIEW_K_AVG, DA2_VIEW_Q_MAX, DA2_VIEW_K_MAX,
@@ -232,11 +237,12 @@ int da2_debug_view(const da2_problem* p, void* ws, int which, void** ptr, size_t
 int da2_rank_noalloc(const da2_problem* p, const float* scores, uint8_t* map, uint16_t* lists,
                      int32_t* counts, void* stream);
 
-/* Device status of the last da2_attention on `ws`: synchronises `stream`, reads
- * the workspace status word and returns DA2_OK, or DA2_ERR_TIMEOUT if a
- * bounded wait inside the attention kernel expired (the call's output is then
- * incomplete), or DA2_ERR_CUDA if the stream reports an error.  No counterpart
- * on the pages: it reports this implementation's own wait bounds. */
+/* Device status of the last da2_prepare and da2_attention on `ws`: synchronises
+ * `stream`, reads the workspace's two status words and returns DA2_OK, or
+ * DA2_ERR_TIMEOUT if a bounded wait inside the V preparation or the attention
+ * kernel expired (the output is then incomplete), or DA2_ERR_CUDA if the
+ * stream reports an error.  No counterpart on the pages: it reports this
+ * implementation's own wait bounds. */
 int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void* stream);
 
 /* Host-buffer form of the whole path (da2_prepare, da2_draft_rank and

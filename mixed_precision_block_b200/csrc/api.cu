@@ -108,7 +108,7 @@ int host_plan(const da2_problem* p, int heads_per_chunk, HostPlan* hp) {
   hp->ws = Lc.total;
   hp->status_off = Lc.off[R_STATUS];
   hp->set = 4 * hp->chunk + hp->ws;
-  hp->status = ((size_t)hp->nchunks * sizeof(int) + 255) & ~(size_t)255;
+  hp->status = ((size_t)hp->nchunks * 2 * sizeof(int) + 255) & ~(size_t)255;  // two status words per chunk
   return DA2_OK;
 }
 
@@ -260,12 +260,13 @@ int da2_check_status(const da2_problem* p, const void* ws, size_t ws_bytes, void
   if (rc) return rc;
   const Layout L = make_layout(g);
   if (!ws || ws_bytes < L.total) return DA2_ERR_WORKSPACE;
-  int word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, static_cast<const char*>(ws) + L.off[R_STATUS], sizeof(int),
+  // word 0: the attention kernel's, word 1: the preparation's
+  int word[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(word, static_cast<const char*>(ws) + L.off[R_STATUS], sizeof(word),
                                   cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  return word ? DA2_ERR_TIMEOUT : DA2_OK;
+  return (word[0] | word[1]) ? DA2_ERR_TIMEOUT : DA2_OK;
 }
 
 int da2_host_bytes(const da2_problem* p, int heads_per_chunk, size_t* bytes) {
@@ -321,8 +322,8 @@ int da2_forward_host(const da2_problem* p, const void* q, const void* k, const v
         (rc = da2_draft_rank(&pcc, ws, hp.ws, cs)) == DA2_OK)
       rc = da2_attention(&pcc, dq, dk, dv, ws, hp.ws, dout, cs);
     if (rc != DA2_OK) break;
-    // the chunk's bounded-wait status (the next use of the workspace clears it)
-    e = cudaMemcpyAsync(status + c, ws + hp.status_off, sizeof(int), cudaMemcpyDeviceToDevice, cs);
+    // the chunk's bounded-wait status words (the next use of the workspace clears them)
+    e = cudaMemcpyAsync(status + 2 * c, ws + hp.status_off, 2 * sizeof(int), cudaMemcpyDeviceToDevice, cs);
     if (e == cudaSuccess) e = cudaEventRecord(ev[1][s], cs);
     // copy out
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev[1][s], 0);
@@ -334,9 +335,9 @@ int da2_forward_host(const da2_problem* p, const void* q, const void* k, const v
   if (e == cudaSuccess) e = e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3);
   if (e == cudaSuccess && rc == DA2_OK) {
     for (int c = 0; c < hp.nchunks && e == cudaSuccess; ++c) {
-      int word = 0;
-      e = cudaMemcpy(&word, status + c, sizeof(int), cudaMemcpyDeviceToHost);
-      if (word) rc = DA2_ERR_TIMEOUT;
+      int word[2] = {0, 0};
+      e = cudaMemcpy(word, status + 2 * c, sizeof(word), cudaMemcpyDeviceToHost);
+      if (word[0] | word[1]) rc = DA2_ERR_TIMEOUT;
     }
   }
   for (int i = 0; i < 3; ++i)

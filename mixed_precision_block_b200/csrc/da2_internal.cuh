@@ -84,7 +84,7 @@ inline Layout make_layout(const Geom& g) {
   L.size[R_MAP] = bh * nb * nb;
   L.size[R_LISTS] = bh * nb * nb * 2;
   L.size[R_COUNTS] = bh * nb * 4 * 4;
-  L.size[R_V_AMAX] = bh * d * 4;
+  L.size[R_V_AMAX] = bh * d * 4 + (bh + 1) * 4;  // absmax bits, work counter, done counter per head
   L.size[R_LOGB] = bh * nb * nb * 4;
   L.size[R_HIST] = (size_t)kRankPasses * bh * kTargets * 256 * 4;
   L.size[R_RSTATE] = bh * kTargets * sizeof(RankState);

@@ -11,10 +11,10 @@
 //   max (warp-shuffle + shared-memory reductions), the INT8 codes with the
 //   block's absmax scale, and the NVFP4 codes with one e4m3 scale per 16
 //   channels of a token.
-// v_amax + pack_v_tma: the per-channel absmax of V over all real tokens of a
-//   head (first pass, atomicMax on the float bits), then the same TMA ring
-//   over V's region tiles, which writes INT8 and NVFP4 codes in
-//   [block][channel][token] order.
+// v_prep: V's per-channel absmax over all real tokens of a head (atomicMax
+//   on the float bits) and, once a head's absmax is complete, the same TMA ring
+//   over V's region tiles writing the INT8 and NVFP4 codes — one persistent
+//   kernel that orders its work so that V crosses HBM once (see v_prep_kernel).
 #include "da2_internal.cuh"
 #include "sm100.cuh"
 
@@ -78,6 +78,7 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t x0, uint32_t x1, uint32_
 // the frame), and the CTA computes from shared memory what prep_qk computes
 // from registers.
 constexpr int kPrepStages = 4;
+constexpr uint32_t kPrepSpin = 1u << 22;  // bound of every wait (polls)
 
 template <int D>
 struct PrepTmaLayout {
@@ -245,48 +246,9 @@ __global__ void __launch_bounds__(kThreads) prep_qk_tma_kernel(const __grid_cons
   }
 }
 
-// Per-channel absmax of V over all real tokens of one head.
-template <int D>
-__global__ void __launch_bounds__(kThreads) v_amax_kernel(Geom g, const __nv_bfloat16* __restrict__ v,
-                                                          unsigned int* __restrict__ amax_bits,
-                                                          int tokens_per_cta) {
-  constexpr int CPT = D / 8;
-  constexpr int ROWS = kThreads / CPT;
-  const int bh = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int cg = tid % CPT;
-  const int t0 = blockIdx.x * tokens_per_cta;
-  const int t1 = min(g.N, t0 + tokens_per_cta);
-  const __nv_bfloat16* __restrict__ x = v + (size_t)bh * g.N * D;
-  float m[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) m[c] = 0.f;
-  for (int t = t0 + tid / CPT; t < t1; t += ROWS) {
-    float f[8];
-    unpack8(*reinterpret_cast<const uint4*>(x + (size_t)t * D + cg * 8), f);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], fabsf(f[c]));
-  }
-#pragma unroll
-  for (int o = CPT; o < 32; o <<= 1)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], __shfl_xor_sync(0xffffffffu, m[c], o));
-  __shared__ float s_m[kThreads / 32][D];
-  if (lane < CPT)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) s_m[warp][cg * 8 + c] = m[c];
-  __syncthreads();
-  if (tid < D) {
-    float r = 0.f;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) r = fmaxf(r, s_m[w][tid]);
-    atomicMax(amax_bits + (size_t)bh * D + tid, __float_as_uint(r));  // r >= 0: bit order = value order
-  }
-}
-
 struct VPtrs {
   const __nv_bfloat16* v;
-  const unsigned int* amax_bits;
+  unsigned int* amax_bits;  // per head and channel: absmax float bits (merged by atomicMax)
   __nv_bfloat16* q8;  // INT8 codes as bf16 values, [block][slot][channel]
   float* s8;
   uint8_t* f4;
@@ -294,14 +256,38 @@ struct VPtrs {
   float* g4;
 };
 
-// pack_v_tma: persistent form of pack_v with the same TMA ring as
-// prep_qk_tma.  The tile stays as loaded ([slot][channel], bf16); a thread
-// takes two neighbouring channels of one 16-slot group, reads them down the
-// slots (a warp covers 64 channels: conflict-free) and writes both channels'
-// INT8 codes and NVFP4 microblock in [block][channel][slot] order.
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// v_prep: V in one pass over HBM.  A head's INT8 and NVFP4 channel scales need
+// the absmax of every channel over all of the head's tokens before any code is
+// written.  So the persistent CTAs take work items from a global counter in
+// the order A(0), B(0), A(1), B(1), ..., where A(h) and B(h) hold one item per
+// V block of head h.  An A(h) item takes the
+// block's channel absmax into the CTA's running absmax of head h, which the
+// CTA merges into the head's (atomicMax on the float bits) and counts as done
+// when it moves to another head's A items, runs out of items, or is about to
+// wait for a head h' >= h.  A B(h) item writes the block's codes once all of
+// head h's A items are counted (a bounded wait: the CTAs still on head h's
+// last A items).  Head h's V tiles were read just before and are still in L2
+// (126 MB against 30 MB per head), so DRAM sees V once.  (Handing out A(h+1)
+// between A(h) and B(h), to hide that wait, let a third of V drop out of L2.)
+// The waits end, by induction on the head: an A item never waits, so a CTA
+// holding unmerged A(h) items waits only for heads before h, which end by the
+// induction; it then reaches its next A head, B(h' >= h) or the end of the
+// items, and merges.  (Keeping A(h) unmerged while waiting for a later head
+// can deadlock: that head's A items may sit behind waits for head h.)  The tile stays as loaded ([slot][channel],
+// bf16); a thread takes two neighbouring channels of one 16-slot group, reads
+// them down the slots (a warp covers 64 channels: conflict-free).
 template <int D>
-__global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_constant__ CUtensorMap tmV, Geom g,
-                                                              VPtrs P, int want_i8, int want_f4, int n_items) {
+__global__ void __launch_bounds__(kThreads) v_prep_kernel(const __grid_constant__ CUtensorMap tmV, Geom g, VPtrs P,
+                                                          int want_i8, int want_f4, int n_items,
+                                                          unsigned int* __restrict__ work,
+                                                          unsigned int* __restrict__ done, int* __restrict__ status,
+                                                          uint32_t spin) {
   using LY = PrepTmaLayout<D>;
   static_assert(D / 2 * 4 == kThreads || D / 2 * 4 == kThreads / 2, "one or half a unit per thread");
   constexpr int UNITS = D / 2 * 4;  // (channel pair, 16-slot group)
@@ -310,13 +296,45 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
   const int tid = threadIdx.x;
   auto bar = [&](int i) { return s0 + LY::BAR + 8u * (uint32_t)i; };
   int4* info = reinterpret_cast<int4*>(psm + LY::INFO);
+  float* s_red = reinterpret_cast<float*>(psm + LY::SUM);       // [4 slot groups][D] absmax partials
+  volatile int* s_go = reinterpret_cast<volatile int*>(psm + LY::AMAX);
   const int t_of = g.nry * g.nrx;
-  auto issue = [&](int item, int stage) {
-    const int bh = item / g.nb, blk = item - bh * g.nb;
+  // item -> (pack, head, block) in the order A(0), B(0), A(1), B(1), ...
+  auto decode = [&](int item, int& is_b, int& bh, int& blk) {
+    const int grp = item / g.nb;
+    blk = item - grp * g.nb;
+    bh = grp >> 1;
+    is_b = grp & 1;
+  };
+  // this CTA's running absmax of head acc_bh over acc_n A items, not yet merged
+  float* s_acc = reinterpret_cast<float*>(psm + LY::MAX);
+  int acc_bh = -1, acc_n = 0;
+  auto flush = [&]() {
+    if (acc_n == 0) return;
+    if (tid < D) {
+      atomicMax(P.amax_bits + (size_t)acc_bh * D + tid, __float_as_uint(s_acc[tid]));  // >= 0: bit order = value order
+      __threadfence();
+    }
+    __syncthreads();  // the merges are visible before the items count as done
+    if (tid == 0) atomicAdd(done + acc_bh, (unsigned int)acc_n);
+    acc_n = 0;
+    acc_bh = -1;
+  };
+  // the issuing thread takes the next item and loads its V tile into `stage`,
+  // or marks the stage empty once the items are exhausted
+  auto issue = [&](int stage) {
+    const int item = (int)atomicAdd(work, 1u);
+    const uint32_t fb = bar(stage);
+    if (item >= n_items) {
+      info[stage] = make_int4(-1, 0, 0, 0);
+      sm100::mbar_arrive(fb);
+      return;
+    }
+    int is_b, bh, blk;
+    decode(item, is_b, bh, blk);
     const int t = blk / t_of, rem = blk - t * t_of;
     const int ry = rem / g.nrx, rx = rem - ry * g.nrx;
-    info[stage] = make_int4(bh, blk, 0, 0);
-    const uint32_t fb = bar(stage);
+    info[stage] = make_int4(is_b, bh, blk, 0);
     sm100::mbar_expect_tx(fb, (uint32_t)LY::STAGE);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c)
@@ -326,24 +344,23 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
     for (int s = 0; s < kPrepStages; ++s) sm100::mbar_init(bar(s), 1);
     sm100::fence_mbar_init();
     sm100::prefetch_tmap(&tmV);
-    for (int s = 0; s < kPrepStages; ++s) {
-      const int item = blockIdx.x + s * gridDim.x;
-      if (item < n_items) issue(item, s);
-    }
+    for (int s = 0; s < kPrepStages; ++s) issue(s);
   }
   __syncthreads();
   const int cp = tid % (D / 2), j = tid / (D / 2);  // channel pair, 16-slot group
   const int c0 = 2 * cp;
   const bool active = tid < UNITS;
   for (int k = 0;; ++k) {
-    const int item = blockIdx.x + k * gridDim.x;
-    if (item >= n_items) break;
     const int stage = k % kPrepStages;
     // bounded wait, agreed by the whole CTA so that no thread leaves alone
-    if (!__syncthreads_and(sm100::mbar_wait(bar(stage), (uint32_t)(k / kPrepStages) & 1u))) break;
+    if (!__syncthreads_and(sm100::mbar_wait(bar(stage), (uint32_t)(k / kPrepStages) & 1u, spin))) {
+      if (tid == 0) atomicOr(status, 1);
+      break;
+    }
     const int4 inf = info[stage];
-    const int bh = inf.x, blk = inf.y;
-    const size_t blk_lin = (size_t)bh * g.nb + blk;
+    // items are taken in increasing order, so the first empty stage comes after every loaded one
+    if (inf.x < 0) break;
+    const int is_b = inf.x, bh = inf.y, blk = inf.z;
     float f0[16], f1[16];
     if (active) {
       const uint8_t* col = psm + stage * LY::STAGE + (c0 >> 6) * LY::BOX + (c0 & 63) * 2;
@@ -356,24 +373,56 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
       }
     }
     __syncthreads();  // every thread has its values: the stage may be refilled
-    if (tid == 0) {
-      const int nxt = blockIdx.x + (k + kPrepStages) * gridDim.x;
-      if (nxt < n_items) issue(nxt, stage);
+    if (tid == 0) issue(stage);
+    if (!is_b) {
+      // ---- A: the block's channel absmax (padding slots hold the TMA zero fill) into the CTA's running one
+      if (acc_bh != bh) flush();
+      if (active) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) { a0 = fmaxf(a0, fabsf(f0[e])); a1 = fmaxf(a1, fabsf(f1[e])); }
+        s_red[j * D + c0] = a0;
+        s_red[j * D + c0 + 1] = a1;
+      }
+      __syncthreads();
+      if (tid < D) {
+        float r = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) r = fmaxf(r, s_red[q * D + tid]);
+        s_acc[tid] = acc_n == 0 ? r : fmaxf(s_acc[tid], r);
+      }
+      acc_bh = bh;
+      ++acc_n;
+      continue;
     }
+    // ---- B: once every A item of the head is done, the codes
+    if (acc_n > 0 && acc_bh <= bh) flush();  // never wait for a head while holding unmerged A items of it or of an earlier head
+    if (tid == 0) {
+      bool ok = *reinterpret_cast<volatile int*>(status) == 0;
+      uint32_t i = 0;
+      while (ok && ld_acquire(done + bh) < (unsigned int)g.nb) {
+        if (++i > spin) { ok = false; atomicOr(status, 1); }
+        __nanosleep(64);
+      }
+      *s_go = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!*s_go) continue;  // a wait gave up: the status word says so; the ring still drains
+    const size_t blk_lin = (size_t)bh * g.nb + blk;
     const unsigned int* amax_bits = P.amax_bits + (size_t)bh * D;
     if (blk == 0 && tid < D) {
-      const float a = __uint_as_float(amax_bits[tid]);
+      const float a = __uint_as_float(__ldcg(amax_bits + tid));
       if (want_i8) P.s8[(size_t)bh * D + tid] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
       if (want_f4) P.g4[(size_t)bh * D + tid] = __fdiv_rn(a, 2688.0f);
     }
     if (!active) continue;
+    const float am0 = __uint_as_float(__ldcg(amax_bits + c0)), am1 = __uint_as_float(__ldcg(amax_bits + c0 + 1));
     if (want_i8) {
       // the codes of channels c0, c0+1 for this thread's 16 slots, as bf16
       // values (integers up to 127: exact), in the block's [slot][channel]
       // order — the layout of a bf16 V tile, so the INT8 phase's P·V runs on
       // the same tensor-core path as the 16-bit phase's
-      const float a0 = __uint_as_float(amax_bits[c0]), a1 = __uint_as_float(amax_bits[c0 + 1]);
-      const float inv0 = a0 > 0.f ? __fdiv_rn(127.0f, a0) : 0.f, inv1 = a1 > 0.f ? __fdiv_rn(127.0f, a1) : 0.f;
+      const float inv0 = am0 > 0.f ? __fdiv_rn(127.0f, am0) : 0.f, inv1 = am1 > 0.f ? __fdiv_rn(127.0f, am1) : 0.f;
       __nv_bfloat16* dst = P.q8 + (blk_lin * 64 + 16 * j) * D + c0;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -383,13 +432,12 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
             __floats2bfloat162_rn((float)k0, (float)k1);
       }
     }
+    if (want_f4) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float* f = h ? f1 : f0;
-      const int c = c0 + h;
-      const float a = __uint_as_float(amax_bits[c]);
-      if (want_f4) {
-        const float gch = __fdiv_rn(a, 2688.0f);
+      for (int h = 0; h < 2; ++h) {
+        float* f = h ? f1 : f0;
+        const int c = c0 + h;
+        const float gch = __fdiv_rn(h ? am1 : am0, 2688.0f);
         const float r = gch > 0.f ? __fdiv_rn(1.0f, gch) : 0.f;
         float a16 = 0.f;
         float y[16];
@@ -404,6 +452,7 @@ __global__ void __launch_bounds__(kThreads) pack_v_tma_kernel(const __grid_const
       }
     }
   }
+  flush();  // the last head's A items, if the items ran out after them
 }
 
 template <int D>
@@ -437,33 +486,34 @@ cudaError_t launch_prepare_d(const Geom& g, const Layout& L, const void* q, cons
     return cudaErrorNotSupported;  // no tensor-map encoder in this driver
   }
   e = cudaGetLastError();
+  // the preparation's status word is cleared by every call, V packed or not
+  int* status = at<int>(ws, L, R_STATUS) + 1;
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (e != cudaSuccess || !(want_i8 || want_f4)) return e;
 
+  // the absmax words, then the work counter and one done counter per head (zero)
   unsigned int* amax = at<unsigned int>(ws, L, R_V_AMAX);
+  unsigned int* work = amax + (size_t)g.BH * D;
+  unsigned int* done = work + 1;
   e = cudaMemsetAsync(amax, 0, L.size[R_V_AMAX], st);
   if (e != cudaSuccess) return e;
-  const int tpc = 2048;
-  v_amax_kernel<D><<<dim3((g.N + tpc - 1) / tpc, g.BH), kThreads, 0, st>>>(
-      g, static_cast<const __nv_bfloat16*>(v), amax, tpc);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (2LL * g.BH * g.nb > 0x7fffffffLL) return cudaErrorNotSupported;
   VPtrs V{static_cast<const __nv_bfloat16*>(v), amax, at<__nv_bfloat16>(ws, L, R_V_I8),
           at<float>(ws, L, R_V_S8), at<uint8_t>(ws, L, R_V_F4), at<uint8_t>(ws, L, R_V_SF4),
           at<float>(ws, L, R_V_G4)};
   CUtensorMap tv;
-  if (make_region_map(&tv, v, g, false)) {
-    using LY = PrepTmaLayout<D>;
-    e = cudaFuncSetAttribute(pack_v_tma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::TOTAL);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_v_tma_kernel<D>, kThreads, LY::TOTAL);
-    const int n_items = g.BH * g.nb;
-    const int grid = std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
-    pack_v_tma_kernel<D><<<grid, kThreads, LY::TOTAL, st>>>(tv, g, V, want_i8, want_f4, n_items);
-  } else {
-    return cudaErrorNotSupported;  // no tensor-map encoder in this driver
-  }
+  if (!make_region_map(&tv, v, g, false)) return cudaErrorNotSupported;  // no tensor-map encoder in this driver
+  using LY = PrepTmaLayout<D>;
+  e = cudaFuncSetAttribute(v_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::TOTAL);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v_prep_kernel<D>, kThreads, LY::TOTAL);
+  const int n_items = 2 * g.BH * g.nb;
+  const int grid = std::max(1, std::min(n_items, sms * std::max(per_sm, 1)));
+  v_prep_kernel<D><<<grid, kThreads, LY::TOTAL, st>>>(tv, g, V, want_i8, want_f4, n_items, work, done, status,
+                                                      kPrepSpin);
   return cudaGetLastError();
 }
 

@@ -47,7 +47,8 @@ def _full_check(wl, heads=None, dense_ref=True):
         if dense_ref:
             dn = PT.dense_rows(qh, kh, vh, toks)
             outs.append(PT.rel_l2(got, dn))
-    assert int(da2.view(p, ws, "STATUS")[0]) == 0
+    st = da2.view(p, ws, "STATUS")
+    assert int(st[0]) == 0 and int(st[1]) == 0  # attention's and the V preparation's bounded waits
     assert da2.da2_check_status(p, ws) == 0
     return outs
 
