@@ -118,11 +118,12 @@ int da2_rank_from_scores(const da2_problem* p, const float* scores, void* ws,
  * Per query block one pass runs the 16-bit phase (bf16 Q/K/V), the INT8 phase
  * and the NVFP4 phase over its assigned key blocks with one shared online
  * softmax state and one fp32 output accumulator.  Low-bit P is quantised per
- * (query row, key block) against that block's own row maximum: INT8 codes
- * round(255 exp(s - m_blk)); NVFP4 of 2688 * 2^(x - ceil(max x)) per 16 keys
- * (x = s log2 e).  Each low-bit block enters numerator and row sum with the
- * same quantised weights, and each phase joins the shared accumulator with
- * its V channel scale.  The output rows are written straight back to the
+ * (query row, key block) against that block's own row maximum rounded up to
+ * a power of two, r = ceil(max x) over the block's real keys (x = s log2 e):
+ * INT8 codes round(255 * 2^(x - r)); NVFP4 of 2688 * 2^(x - r) per 16 keys.
+ * Each low-bit block enters numerator and row sum with the same quantised
+ * weights, and each phase joins the shared accumulator with its V channel
+ * scale.  The output rows are written straight back to the
  * original token order (padding rows dropped); a query block with no key
  * block outputs zeros.
  * q, k, v: the same device tensors given to da2_prepare; out: device bf16
