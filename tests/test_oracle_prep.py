@@ -1,4 +1,4 @@
-"""Pins for the oracle's V preparation and its plain dense attention (CPU only).
+"""Pins for the oracle's Q/K and V quantisers and its plain dense attention (CPU only).
 
 V's INT8 codes are checked through the invariants of a symmetric per-channel
 quantiser rather than by recomputing its formula: the channel's largest
@@ -7,8 +7,10 @@ all-zero channel gives scale 0, and padding slots hold code 0.  NVFP4 V is
 checked by an exact round trip of values built on the format's grid with a
 different microscale for every (channel, 16-token group): that fails if the
 microblocks ran along channels instead of along the tokens (the reduction axis
-of P·V), or if the per-channel outer scale were off.  The dense attention is
-checked against torch's fp64 scaled-dot-product attention.
+of P·V), or if the per-channel outer scale were off.  Q and K the same way:
+one INT8 scale per 64-token block, NVFP4 microblocks along 16 channels of a
+token.  The dense attention is checked against torch's fp64
+scaled-dot-product attention.
 """
 
 import numpy as np
@@ -83,3 +85,39 @@ def test_dense_attention_matches_torch_sdpa():
         want = torch.nn.functional.scaled_dot_product_attention(
             *(torch.from_numpy(x)[None, None] for x in (q, k, v)))[0, 0].numpy()
         np.testing.assert_allclose(OA.dense_attention(q, k, v), want, rtol=1e-12, atol=1e-12)
+
+
+def test_qk_int8_one_scale_per_block():
+    rng = np.random.default_rng(8)
+    n, d = 100, 16
+    x = rng.normal(size=(n, d)).astype(np.float32).astype(np.float64)
+    x[70:, :] *= 0.01  # the second block is much smaller: its own scale keeps its resolution
+    blocks, valid = OP.gather_blocks(x, _table(n, 2))
+    codes, scale = OP.qk_int8(blocks)
+    assert codes.shape == (2, 64, d) and scale.shape == (2,)
+    for b in range(2):
+        amax = np.abs(blocks[b][valid[b]]).max()
+        np.testing.assert_allclose(scale[b] * 127.0, amax, rtol=2e-7)
+        assert np.abs(codes[b].astype(np.int64)).max() == 127
+        err = np.abs(codes[b].astype(np.float64) * scale[b] - blocks[b])[valid[b]]
+        assert np.all(err <= 0.5 * scale[b] * (1 + 1e-5) + 1e-12)
+    assert np.all(codes[~valid] == 0)
+
+
+def test_qk_nvfp4_round_trips_on_its_grid_along_channels():
+    rng = np.random.default_rng(9)
+    d = 64
+    e2m1_vals = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    e4m3_vals = np.unique(np.abs(F.e4m3_decode(np.arange(256))))
+    e4m3_vals = e4m3_vals[np.isfinite(e4m3_vals) & (e4m3_vals >= 2.0 ** -6) & (e4m3_vals <= 448.0)]
+    x = np.zeros((64, d))
+    for t in range(64):
+        for j in range(d // 16):  # one microscale per (token, 16 consecutive channels)
+            s = float(rng.choice(e4m3_vals))
+            vals = rng.choice(e2m1_vals, 16) * rng.choice([-1.0, 1.0], 16)
+            vals[rng.integers(16)] = 6.0 * rng.choice([-1.0, 1.0])
+            x[t, 16 * j:16 * j + 16] = s * vals
+    blocks, _ = OP.gather_blocks(x, _table(64, 1))
+    codes, sf = OP.qk_nvfp4(blocks)
+    assert codes.shape == (1, 64, d) and sf.shape == (1, 64, d // 16)
+    np.testing.assert_array_equal(F.nvfp4_dequantize(codes, sf), blocks)
