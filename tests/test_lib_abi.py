@@ -122,19 +122,20 @@ def test_status_strings(da2):
 
 
 def test_host_path_sizes_and_argument_checks(da2):
-    # two sets of (Q, K, V, O chunk + chunk workspace) plus one status word per
-    # chunk; a chunk of G heads is the same problem with B = 1, H = G
-    wl = WORKLOADS["mid"]
-    p = da2.Problem.from_workload(wl)
-    info = da2.da2_plan(p)
-    for G in (1, 5, 12, 40):
-        Gc = min(G, wl.B * wl.H)
-        pc = da2.Problem.from_workload(wl, B=1, H=Gc)
-        chunk = -(-info.N * wl.d * 2 * Gc // 256) * 256
-        nchunks = -(-(wl.B * wl.H) // Gc)
-        status = -(-nchunks * 4 // 256) * 256
-        want = 2 * (4 * chunk + da2.da2_plan(pc).ws_bytes) + status
-        assert da2.da2_host_bytes(p, G) == want
+    # two sets of (Q, K, V, O chunk + chunk workspace) plus two status words
+    # per chunk (the attention kernel's and the V preparation's); a chunk of G
+    # heads is the same problem with B = 1, H = G
+    for wl, Gs in ((WORKLOADS["mid"], (1, 5, 12, 40)), (WORKLOADS["mid"].with_(H=100), (1, 3))):
+        p = da2.Problem.from_workload(wl)
+        info = da2.da2_plan(p)
+        for G in Gs:
+            Gc = min(G, wl.B * wl.H)
+            pc = da2.Problem.from_workload(wl, B=1, H=Gc)
+            chunk = -(-info.N * wl.d * 2 * Gc // 256) * 256
+            nchunks = -(-(wl.B * wl.H) // Gc)
+            status = -(-nchunks * 8 // 256) * 256  # 100 chunks: 1024 bytes, not 512
+            want = 2 * (4 * chunk + da2.da2_plan(pc).ws_bytes) + status
+            assert da2.da2_host_bytes(p, G) == want
     with pytest.raises(da2.Da2Error) as e:
         da2.da2_host_bytes(p, 0)
     assert e.value.code == da2.DA2_ERR_ARG
